@@ -1,0 +1,339 @@
+"""Pins that tie the fp64 oracle to something other than itself.
+
+Each pin is a function ``pin_xxx(orc)`` that raises ``AssertionError`` when the
+oracle ``orc`` is wrong.  They are run twice: against the real oracle (all must
+pass) and against builds with one planted mistake each (at least one must
+fail), so a plausible slip -- a wrong head map, a swapped page/row index, a
+dropped scale or normaliser, an off-by-one causal edge, the wrong cache layout,
+a flipped merge sign -- cannot hide.
+
+What pins what (the method: paged gather through a block table, Tiny-Infer page
+section "分页KV缓存：借鉴操作系统的内存管理"; exact softmax attention,
+"5 Fun Projects for LLM Inference Engineering" section 2):
+
+* closed-form golden cases (tests/golden) -- hand-derived softmax values;
+* brute force -- an independent NumPy full-matrix formulation;
+* paged == contiguous -- a static cache written into shuffled pages by the
+  oracle's own scatter gives bit-identical results;
+* scatter/gather identity, skip of negative slots, rejection of slots outside
+  the pool;
+* single key -> its V row; identical keys -> mean of V; scale 0 -> mean of V;
+* one-hot V exposes the probability row: it sums to 1 and matches exp/sum;
+* causal: future keys do not matter; the last query of a chunk equals decode;
+* GQA equals materialised MHA; G = 1 is plain MHA;
+* split-KV partials merged by log-sum-exp equal the plain result;
+* an empty context gives a zero row.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+
+from oracle import bf16_bits_to_f64
+from oracle import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "closed_form_cases.json")
+
+
+# --------------------------------------------------------------------------- #
+# small helpers (numpy only; bf16 values as uint16 bit patterns)               #
+# --------------------------------------------------------------------------- #
+
+def f32_to_bf16_bits(x) -> np.ndarray:
+    """Round float values to bf16 (round to nearest even) and return the bits."""
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def rand_bits(rng, shape, std=1.0):
+    return f32_to_bf16_bits(rng.standard_normal(shape) * std)
+
+
+def make_paged(rng, lens, Hkv, D, bs, extra_blocks=3):
+    """Random paged pool for the given lengths; NaN in every unused slot."""
+    pages = [-(-L // bs) for L in lens]
+    NB = sum(pages) + extra_blocks
+    perm = rng.permutation(NB)
+    MB = max(pages + [1])
+    bt = np.full((len(lens), MB), -1, dtype=np.int32)
+    off = 0
+    for b, p in enumerate(pages):
+        bt[b, :p] = perm[off:off + p]
+        off += p
+    k = rand_bits(rng, (NB, Hkv, bs, D))
+    v = rand_bits(rng, (NB, Hkv, bs, D))
+    valid = np.zeros((NB, bs), dtype=bool)
+    for b, L in enumerate(lens):
+        for j in range(L):
+            valid[bt[b, j // bs], j % bs] = True
+    bad = np.broadcast_to((~valid)[:, None, :, None], k.shape)
+    k[bad] = 0x7FC0
+    v[bad] = 0x7FC0
+    return k, v, bt, np.asarray(lens, dtype=np.int32)
+
+
+def scatter_contiguous(orc, kc, vc, lens, bs, rng, extra_blocks=2):
+    """Write a contiguous [B, Lmax, Hkv, D] cache into shuffled pages using the
+    oracle's own cache write; returns (k_cache, v_cache, block_tables)."""
+    B, Lmax, Hkv, D = kc.shape
+    pages = [-(-int(L) // bs) for L in lens]
+    NB = sum(pages) + extra_blocks
+    perm = rng.permutation(NB)
+    MB = max(pages + [1])
+    bt = np.full((B, MB), -1, dtype=np.int32)
+    off = 0
+    for b, p in enumerate(pages):
+        bt[b, :p] = perm[off:off + p]
+        off += p
+    k_cache = np.full((NB, Hkv, bs, D), 0x7FC0, dtype=np.uint16)
+    v_cache = np.full((NB, Hkv, bs, D), 0x7FC0, dtype=np.uint16)
+    for b in range(B):
+        L = int(lens[b])
+        if L == 0:
+            continue
+        slots = np.array([bt[b, j // bs] * bs + j % bs for j in range(L)], dtype=np.int64)
+        orc.kv_cache_write(np.ascontiguousarray(kc[b, :L]), np.ascontiguousarray(vc[b, :L]),
+                           k_cache, v_cache, slots)
+    return k_cache, v_cache, bt
+
+
+# --------------------------------------------------------------------------- #
+# pins                                                                         #
+# --------------------------------------------------------------------------- #
+
+def pin_golden_closed_form(orc):
+    cases = json.load(open(GOLDEN))["cases"]
+    rng = np.random.default_rng(7)
+    for c in cases:
+        keys = np.asarray(c["keys"], dtype=np.float32)
+        vals = np.asarray(c["values"], dtype=np.float32)
+        q = np.asarray(c["q"], dtype=np.float32)
+        L, D = keys.shape
+        Q = q.shape[0]
+        assert c["query_positions"] == list(range(L - Q, L))
+        kb, vb = f32_to_bf16_bits(keys), f32_to_bf16_bits(vals)
+        assert np.array_equal(bf16_bits_to_f64(kb), keys.astype(np.float64)), "inputs must be bf16-exact"
+        bs = 2
+        kc, vc, bt = scatter_contiguous(orc, kb[None, :, None, :], vb[None, :, None, :], [L], bs, rng)
+        qb = f32_to_bf16_bits(q)[:, None, :]                      # [Q, 1, D]
+        expected = np.asarray(c["expected"], dtype=np.float64)
+        out = orc.paged_attention_prefill(qb, np.array([0, Q], np.int32), kc, vc, bt,
+                                          np.array([L], np.int32), c["scale"])
+        np.testing.assert_allclose(out[:, 0, :], expected, rtol=0, atol=1e-15, err_msg=c["name"])
+        # the last query is a decode over all L keys
+        dec = orc.paged_attention(qb[-1:], kc, vc, bt, np.array([L], np.int32), c["scale"])
+        np.testing.assert_allclose(dec[0, 0], expected[-1], rtol=0, atol=1e-15, err_msg=c["name"])
+
+
+def pin_brute_force_decode(orc):
+    rng = np.random.default_rng(11)
+    for (lens, Hq, Hkv, D, bs) in [([37, 100], 4, 2, 64, 16), ([1, 5, 16, 17, 33], 8, 2, 32, 4),
+                                   ([70, 3], 6, 3, 16, 8), ([20], 4, 4, 8, 16)]:
+        k, v, bt, cl = make_paged(rng, lens, Hkv, D, bs)
+        q = rand_bits(rng, (len(lens), Hq, D))
+        scale = float(np.float32(1.0) / np.sqrt(np.float32(D)))
+        got = orc.paged_attention(q, k, v, bt, cl, scale)
+        ref = brute.paged_attention(q, k, v, bt, cl, scale)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def pin_brute_force_prefill(orc):
+    rng = np.random.default_rng(12)
+    for (lens, qlens, Hq, Hkv, D, bs) in [([40, 19], [7, 19], 4, 2, 32, 16),
+                                          ([9, 33, 1], [9, 5, 1], 6, 2, 16, 4)]:
+        k, v, bt, cl = make_paged(rng, lens, Hkv, D, bs)
+        qsl = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+        q = rand_bits(rng, (int(qsl[-1]), Hq, D))
+        scale = 0.3
+        got = orc.paged_attention_prefill(q, qsl, k, v, bt, cl, scale)
+        ref = brute.paged_attention_prefill(q, qsl, k, v, bt, cl, scale)
+        np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def pin_paged_equals_contiguous(orc):
+    rng = np.random.default_rng(13)
+    B, Lmax, Hq, Hkv, D, bs = 3, 50, 4, 2, 16, 16
+    lens = np.array([50, 17, 33], dtype=np.int32)
+    kc = rand_bits(rng, (B, Lmax, Hkv, D))
+    vc = rand_bits(rng, (B, Lmax, Hkv, D))
+    q = rand_bits(rng, (B, Hq, D))
+    k_cache, v_cache, bt = scatter_contiguous(orc, kc, vc, lens, bs, rng)
+    paged = orc.paged_attention(q, k_cache, v_cache, bt, lens, 0.25)
+    contig = orc.contiguous_attention(q, kc, vc, lens, 0.25)
+    assert np.array_equal(paged, contig), "paged and contiguous layouts must agree bit for bit"
+
+
+def pin_scatter_gather_identity(orc):
+    rng = np.random.default_rng(14)
+    NB, Hkv, bs, D, T = 6, 2, 4, 8, 9
+    k_cache = rand_bits(rng, (NB, Hkv, bs, D))
+    v_cache = rand_bits(rng, (NB, Hkv, bs, D))
+    k0, v0 = k_cache.copy(), v_cache.copy()
+    key = rand_bits(rng, (T, Hkv, D))
+    val = rand_bits(rng, (T, Hkv, D))
+    slots = rng.permutation(NB * bs)[:T].astype(np.int64)
+    slots[3] = -1                                   # padding token: skipped
+    rc = orc.kv_cache_write(key, val, k_cache, v_cache, slots)
+    assert rc == 0
+    touched = np.zeros((NB, bs), dtype=bool)
+    for t, s in enumerate(slots):
+        if s < 0:
+            continue
+        blk, off = divmod(int(s), bs)
+        touched[blk, off] = True
+        assert np.array_equal(k_cache[blk, :, off, :], key[t])
+        assert np.array_equal(v_cache[blk, :, off, :], val[t])
+    keep = np.broadcast_to((~touched)[:, None, :, None], k_cache.shape)
+    assert np.array_equal(k_cache[keep], k0[keep]), "untouched slots changed"
+    assert np.array_equal(v_cache[keep], v0[keep])
+    # a slot outside the pool is reported and writes nothing
+    k1, v1 = k_cache.copy(), v_cache.copy()
+    rc = orc.kv_cache_write(key[:1], val[:1], k_cache, v_cache,
+                            np.array([NB * bs], np.int64), allow_bounds=True)
+    assert rc == 5 and np.array_equal(k_cache, k1) and np.array_equal(v_cache, v1)
+
+
+def pin_single_key_returns_v(orc):
+    rng = np.random.default_rng(15)
+    k, v, bt, cl = make_paged(rng, [1, 1, 1], 2, 32, 16)
+    q = rand_bits(rng, (3, 4, 32))
+    out = orc.paged_attention(q, k, v, bt, cl, 0.7)
+    for b in range(3):
+        for h in range(4):
+            vrow = bf16_bits_to_f64(v[bt[b, 0], h // 2, 0])
+            assert np.array_equal(out[b, h], vrow)
+
+
+def pin_identical_keys_mean_v(orc):
+    rng = np.random.default_rng(16)
+    L, Hkv, D, bs = 45, 1, 16, 16
+    kc = np.repeat(rand_bits(rng, (1, 1, 1, D)), L, axis=1)
+    vc = rand_bits(rng, (1, L, Hkv, D))
+    q = rand_bits(rng, (1, 2, D))
+    k_cache, v_cache, bt = scatter_contiguous(orc, kc, vc, [L], bs, rng)
+    out = orc.paged_attention(q, k_cache, v_cache, bt, np.array([L], np.int32), 0.125)
+    mean = bf16_bits_to_f64(vc[0, :, 0, :]).mean(axis=0)
+    for h in range(2):
+        np.testing.assert_allclose(out[0, h], mean, rtol=0, atol=1e-14)
+
+
+def pin_scale_zero_mean_v(orc):
+    rng = np.random.default_rng(17)
+    k, v, bt, cl = make_paged(rng, [29], 2, 16, 8)
+    q = rand_bits(rng, (1, 2, 16))
+    out = orc.paged_attention(q, k, v, bt, cl, 0.0)
+    V = brute.dense_kv(v, bt[0], 29)
+    for h in range(2):
+        np.testing.assert_allclose(out[0, h], V[:, h].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def pin_softmax_row_sums_to_one(orc):
+    """With V row j = unit vector e_j the output row IS the probability row."""
+    rng = np.random.default_rng(18)
+    L, D, bs = 24, 32, 8
+    kc = rand_bits(rng, (1, L, 1, D))
+    eye = np.zeros((1, L, 1, D), dtype=np.float32)
+    for j in range(L):
+        eye[0, j, 0, j] = 1.0
+    vc = f32_to_bf16_bits(eye)
+    q = rand_bits(rng, (1, 1, D))
+    k_cache, v_cache, bt = scatter_contiguous(orc, kc, vc, [L], bs, rng)
+    scale = 0.2
+    p = orc.paged_attention(q, k_cache, v_cache, bt, np.array([L], np.int32), scale)[0, 0, :L]
+    assert abs(p.sum() - 1.0) < 1e-13
+    s = np.float64(np.float32(scale)) * (bf16_bits_to_f64(kc[0, :, 0, :]) @ bf16_bits_to_f64(q[0, 0]))
+    w = np.exp(s - s.max())
+    np.testing.assert_allclose(p, w / w.sum(), rtol=1e-13, atol=1e-16)
+
+
+def pin_causal_mask(orc):
+    rng = np.random.default_rng(19)
+    L, Q, Hq, Hkv, D, bs = 40, 12, 4, 2, 16, 8
+    kc = rand_bits(rng, (1, L, Hkv, D))
+    vc = rand_bits(rng, (1, L, Hkv, D))
+    q = rand_bits(rng, (Q, Hq, D))
+    qsl = np.array([0, Q], np.int32)
+    cl = np.array([L], np.int32)
+    k1, v1, bt = scatter_contiguous(orc, kc, vc, [L], bs, np.random.default_rng(5))
+    base = orc.paged_attention_prefill(q, qsl, k1, v1, bt, cl, 0.25)
+    # perturb keys/values after position p: queries at positions <= p unchanged
+    p = L - Q + 4                                   # query index 4 sits at position p
+    kc2, vc2 = kc.copy(), vc.copy()
+    kc2[0, p + 1:] = rand_bits(rng, kc2[0, p + 1:].shape)
+    vc2[0, p + 1:] = rand_bits(rng, vc2[0, p + 1:].shape)
+    k2, v2, bt2 = scatter_contiguous(orc, kc2, vc2, [L], bs, np.random.default_rng(5))
+    pert = orc.paged_attention_prefill(q, qsl, k2, v2, bt2, cl, 0.25)
+    assert np.array_equal(base[:5], pert[:5]), "a query saw a future key"
+    assert not np.array_equal(base[5:], pert[5:]), "later queries must see the change"
+    # the chunk's last query equals decode over all L keys
+    dec = orc.paged_attention(q[-1:], k1, v1, bt, cl, 0.25)
+    assert np.array_equal(dec[0], base[-1])
+
+
+def pin_gqa_equals_materialised_mha(orc):
+    rng = np.random.default_rng(20)
+    B, Lmax, Hq, Hkv, D, bs = 2, 30, 6, 2, 16, 8
+    lens = np.array([30, 11], np.int32)
+    kc = rand_bits(rng, (B, Lmax, Hkv, D))
+    vc = rand_bits(rng, (B, Lmax, Hkv, D))
+    q = rand_bits(rng, (B, Hq, D))
+    G = Hq // Hkv
+    kg, vg, btg = scatter_contiguous(orc, kc, vc, lens, bs, np.random.default_rng(1))
+    gqa = orc.paged_attention(q, kg, vg, btg, lens, 0.3)
+    # materialise: kv head h of the MHA cache is the GQA head h // G (consecutive groups)
+    km, vm, btm = scatter_contiguous(orc, np.repeat(kc, G, axis=2), np.repeat(vc, G, axis=2), lens,
+                                     bs, np.random.default_rng(1))
+    mha = orc.paged_attention(q, km, vm, btm, lens, 0.3)
+    assert np.array_equal(gqa, mha)
+    # two query heads of one group with the same q give the same row
+    q2 = q.copy()
+    q2[:, 1] = q2[:, 0]
+    o2 = orc.paged_attention(q2, kg, vg, btg, lens, 0.3)
+    assert np.array_equal(o2[:, 0], o2[:, 1])
+
+
+def pin_split_merge_equals_plain(orc):
+    rng = np.random.default_rng(21)
+    lens = [100, 1, 64, 0, 37]
+    k, v, bt, cl = make_paged(rng, lens, 2, 16, 16)
+    q = rand_bits(rng, (len(lens), 4, 16))
+    plain = orc.paged_attention(q, k, v, bt, cl, 0.25)
+    for S in (16, 32, 48, 100, 128):
+        C = -(-max(lens) // S)
+        o, lse = orc.decode_partials(q, k, v, bt, cl, 0.25, S, C)
+        merged = orc.lse_merge(o, lse)
+        np.testing.assert_allclose(merged, plain, rtol=0, atol=1e-12)
+    # the merge itself: two halves with known weights
+    o_part = np.array([[[1.0, 0.0], [0.0, 1.0]]])
+    lse = np.array([[np.log(3.0), np.log(1.0)]])
+    np.testing.assert_allclose(orc.lse_merge(o_part, lse), [[0.75, 0.25]], atol=1e-15)
+
+
+def pin_empty_context_is_zero(orc):
+    rng = np.random.default_rng(22)
+    k, v, bt, cl = make_paged(rng, [0, 5], 1, 8, 4)
+    q = rand_bits(rng, (2, 2, 8))
+    out = orc.paged_attention(q, k, v, bt, cl, 1.0)
+    assert np.array_equal(out[0], np.zeros((2, 8)))
+    assert np.isfinite(out[1]).all()
+
+
+ALL_PINS = [
+    pin_golden_closed_form,
+    pin_brute_force_decode,
+    pin_brute_force_prefill,
+    pin_paged_equals_contiguous,
+    pin_scatter_gather_identity,
+    pin_single_key_returns_v,
+    pin_identical_keys_mean_v,
+    pin_scale_zero_mean_v,
+    pin_softmax_row_sums_to_one,
+    pin_causal_mask,
+    pin_gqa_equals_materialised_mha,
+    pin_split_merge_equals_plain,
+    pin_empty_context_is_zero,
+]

@@ -1,0 +1,27 @@
+"""Each planted oracle mistake must be caught by at least one pin (CPU only).
+
+The mutants are compile-time variants of the C oracle (PKV_ORACLE_MUTANT):
+1 interleaved GQA head map, 2 page/row index swapped, 3 scale dropped,
+4 causal edge off by one, 5 newest key dropped in decode, 6 softmax
+normaliser dropped, 7 token-major page layout, 8 cache-write slot off by one,
+9 scores taken against V, 10 merge weight sign flipped.
+"""
+import pytest
+
+import oracle
+import oracle_pins
+
+MUTANTS = list(range(1, 11))
+
+
+@pytest.mark.parametrize("mutant", MUTANTS)
+def test_mutant_is_caught(mutant):
+    orc = oracle.Oracle(mutant=mutant)
+    assert orc.mutant == mutant
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(orc)
+        except Exception:            # AssertionError, or the oracle rejecting its own output
+            caught.append(pin.__name__)
+    assert caught, f"mutant {mutant} passed every pin"
