@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV attention hot path on B200.
+
+One step = one decode step of the Llama-3-8B-shaped batch (B=128, 32 q / 8 kv
+heads, head_dim 128, every context 4096, block_size 16): the cache write of one
+new K/V row per sequence, then decode attention over all pages (split-KV
+partials + log-sum-exp merge when the planner splits).  Metric: algorithmic
+bytes of the step / step time in GB/s (the K/V read is 99.9 % of them), plus
+the decode kernel's roofline fraction of the measured HBM copy bandwidth.
+
+Other workloads (Llama-3.2-1B-shaped decode, ragged long-context decode,
+chunked causal prefill in TFLOP/s) are reported under "extras" after the timed
+region; they are not part of the step.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Multi-GPU (torchrun): every rank runs its own replica of the step on its own
+GPU (the decode batch shards by sequence with no exchange); value = all
+ranks' bytes / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode attn KV-read GB/s (% of HBM peak); prefill TFLOP/s (% of bf16 peak)"
+WORKLOAD = "llama3_8b_decode"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "paged_kv_cache_477_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key: str, src_hash: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source
+    is unchanged since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel_key)
+    if not d or d.get("source_hash") != src_hash:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------------- #
+# clocks during the timed region                                               #
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                smax.append(float(parts[2].split()[0]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# algorithmic bytes / flops                                                    #
+# --------------------------------------------------------------------------- #
+def decode_bytes(case) -> int:
+    kv = case.kv_bytes_read()
+    qo = 2 * case.B * case.Hq * case.D * 2
+    bt = sum(-(-L // case.bs) for L in case.lens) * 4 + case.B * 4
+    return kv + qo + bt
+
+
+def write_bytes(case) -> int:
+    if case.new_key is None:
+        return 0
+    T = case.new_key.shape[0]
+    return 2 * (2 * T * case.Hkv * case.D * 2) + T * 8
+
+
+def prefill_flops(case) -> int:
+    """4 * D per (query, visible key) per q head: QK^T and PV, 2 flop per MAC."""
+    f = 0
+    qsl = case.query_start_loc.cpu().tolist()
+    for b in range(case.B):
+        Q, L = qsl[b + 1] - qsl[b], case.lens[b]
+        vis = sum(L - Q + i + 1 for i in range(Q))
+        f += 4 * case.D * vis * case.Hq
+    return f
+
+
+# --------------------------------------------------------------------------- #
+# the oracle on host cores                                                     #
+# --------------------------------------------------------------------------- #
+def oracle_decode_rate(seconds: float):
+    """Oracle decode over a bounded sample of llama3_8b_decode-shaped sequences.
+    Returns (GB/s, cores, sample description)."""
+    import oracle
+    from paged_kv_cache_477_b200 import workloads as wl
+    from paged_kv_cache_477_b200.workloads import bf16_bits
+    orc = oracle.get()
+    spec = wl.WORKLOADS[WORKLOAD]
+
+    def run(nseq):
+        c = wl.make_case(B=nseq, Hq=spec["Hq"], Hkv=spec["Hkv"], D=spec["D"], bs=spec["bs"],
+                         lens=[spec["lens"][0]] * nseq, seed=spec["seed"], device="cpu")
+        q, k, v = bf16_bits(c.q), bf16_bits(c.k_cache), bf16_bits(c.v_cache)
+        bt, cl = c.block_tables.numpy(), c.context_lens.numpy()
+        t0 = time.perf_counter()
+        orc.paged_attention(q, k, v, bt, cl, c.scale)
+        return time.perf_counter() - t0, decode_bytes(c)
+
+    t1, _ = run(1)
+    n = int(max(1, min(spec["B"], seconds / max(t1, 1e-3))))
+    t, nbytes = run(n)
+    desc = (f"fp64 C oracle decode of {n} of the {spec['B']} sequences (ctx {spec['lens'][0]}, "
+            f"{spec['Hq']} q / {spec['Hkv']} kv heads, D={spec['D']}), OpenMP, {t:.1f} s")
+    return nbytes / t / 1e9, orc.num_threads(), desc, t
+
+
+# --------------------------------------------------------------------------- #
+# reference arm: the oracle, as it stands, on host cores                       #
+# --------------------------------------------------------------------------- #
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    per_step = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_decode_rate(per_step)
+    vals, secs = [], 0.0
+    desc, cores = "", 1
+    for _ in range(args.steps):
+        v, cores, desc, t = oracle_decode_rate(per_step)
+        vals.append(v)
+        secs += t
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD} (bounded sample per step)", "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- #
+# extras (after the timed region)                                              #
+# --------------------------------------------------------------------------- #
+def l2_flush_buffer():
+    return torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+
+def time_calls(fn, iters, flush=None):
+    """Per-call device times (ms) with CUDA events on the current stream."""
+    st = torch.cuda.current_stream()
+    ts = []
+    for _ in range(iters):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        fn()
+        e1.record(st)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return ts
+
+
+def extras(peaks):
+    import paged_kv_cache_477_b200 as pkv
+    from paged_kv_cache_477_b200 import workloads as wl
+    res = {}
+    for name, hint in (("llama32_1b_decode", 4096), ("ragged_long_decode", 32768)):
+        c = wl.workload(name, device="cuda")
+        out = torch.empty_like(c.q)
+        ws = torch.empty(max(1, pkv.workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, hint)),
+                         dtype=torch.uint8, device="cuda")
+        fn = lambda: pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale,
+                                         out=out, max_context_len=hint, workspace=ws)
+        time_calls(fn, 3)
+        ts = time_calls(fn, 20)
+        ms = statistics.median(ts)
+        gbs = decode_bytes(c) / (ms * 1e-3) / 1e9
+        res[name] = {"GB/s": round(gbs, 1), "us": round(ms * 1e3, 2), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                     "launches": pkv.last_launch_count(), "bytes": decode_bytes(c),
+                     "l2": "inputs larger than L2"}
+        del c, out, ws
+        torch.cuda.empty_cache()
+    c = wl.workload("chunked_prefill", device="cuda")
+    pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)
+    out = torch.empty_like(c.q)
+    fn = lambda: pkv.paged_attention_prefill(c.q, c.query_start_loc, c.k_cache, c.v_cache, c.block_tables,
+                                             c.context_lens, c.scale, c.max_q_len, out=out)
+    try:
+        flush = l2_flush_buffer()
+        time_calls(fn, 3, flush)
+        ts = time_calls(fn, 20, flush)
+        ms = statistics.median(ts)
+        tf = prefill_flops(c) / (ms * 1e-3) / 1e12
+        res["chunked_prefill"] = {"TFLOP/s": round(tf, 1), "us": round(ms * 1e3, 2),
+                                  "frac_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+                                  "flops": prefill_flops(c), "l2": "flushed (256 MiB write) before each call"}
+    except pkv.PagedKVError as e:
+        res["chunked_prefill"] = {"unavailable": str(e)}
+    return res
+
+
+# --------------------------------------------------------------------------- #
+# main arm                                                                     #
+# --------------------------------------------------------------------------- #
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import paged_kv_cache_477_b200 as pkv
+    from paged_kv_cache_477_b200 import workloads as wl
+
+    pkv.load_library()
+    peaks = measured_peaks()
+    case = wl.workload(WORKLOAD, device="cuda")
+    hint = max(case.lens)
+    out = torch.empty_like(case.q)
+    ws_bytes = pkv.workspace_size(case.B, case.Hq, case.Hkv, case.D, case.MB, case.bs, hint)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
+    st = torch.cuda.current_stream()
+
+    def step():
+        pkv.kv_cache_write(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping)
+        n = pkv.last_launch_count()
+        pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                            case.scale, out=out, max_context_len=hint, workspace=ws)
+        return n + pkv.last_launch_count()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+
+    # ---- timed region: K steps, events around the attention launches ----------
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches = 0
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0.record(st)
+        for i in range(args.steps):
+            pkv.kv_cache_write(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping)
+            launches += pkv.last_launch_count()
+            ev[i][0].record(st)
+            pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                                case.scale, out=out, max_context_len=hint, workspace=ws)
+            launches += pkv.last_launch_count()
+            ev[i][1].record(st)
+        t1.record(st)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    elapsed_ms = t0.elapsed_time(t1)
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    clocks = clk.summary()
+    attn_launches = pkv.last_launch_count()
+    assert pkv.get_device_error() == 0
+
+    # ---- end to end through the public API with host buffers -----------------
+    host_in = {k: getattr(case, k).cpu().pin_memory() for k in
+               ("q", "new_key", "new_value", "slot_mapping", "block_tables", "context_lens")}
+    dev_in = {k: torch.empty_like(getattr(case, k)) for k in host_in}
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k in host_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        pkv.kv_cache_write(dev_in["new_key"], dev_in["new_value"], case.k_cache, case.v_cache,
+                           dev_in["slot_mapping"])
+        pkv.paged_attention(dev_in["q"], case.k_cache, case.v_cache, dev_in["block_tables"],
+                            dev_in["context_lens"], case.scale, out=out, max_context_len=hint, workspace=ws)
+        host_out.copy_(out, non_blocking=True)
+        st.synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    step_bytes = decode_bytes(case) + write_bytes(case)
+    attn_bytes = decode_bytes(case)
+    if dist is not None:
+        tt = torch.tensor([elapsed_ms, e2e_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = tt.tolist()
+
+    if rank == 0:
+        ms_step = elapsed_ms / args.steps
+        value = world * step_bytes / (ms_step * 1e-3) / 1e9
+        e2e_val = world * step_bytes / (e2e_ms / args.steps * 1e-3) / 1e9
+        achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+        src = source_hash("decode_attn.cuh", "pkv_common.cuh")
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.describe(WORKLOAD), "step": "kv_cache_write (128 rows) + paged_attention",
+                       "bytes_per_step": step_bytes,
+                       "l2": "inputs larger than L2: 2 GiB of K/V read per step, no flush needed",
+                       "parallelism": f"replicas{world}" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "kernel": "decode_attn" + (" + lse_merge" if attn_launches == 2 else ""),
+                         "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
+                         "bytes_per_launch": attn_bytes, "us_per_launch": round(attn_ms * 1e3, 2),
+                         "traffic": profiled_traffic("decode_attn", src)},
+            "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        if not args.no_extras and world == 1:
+            line["extras"] = extras(peaks)
+        if world == 1:
+            v, cores, desc, _ = oracle_decode_rate(args.cpu_seconds)
+            line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                    "sample": desc}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,196 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: attention over a block-paged KV cache
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method (from the pages this library follows):
+ *   - "从零构建CUDA推理引擎：Tiny-Infer项目的技术深度解析", section
+ *     "分页KV缓存：借鉴操作系统的内存管理": the KV cache is divided into
+ *     fixed-size blocks ("pages") and a mapping table turns each logical
+ *     position into a physical block, so sequences can share memory and grow.
+ *   - same page, section "Flash Attention：内存与计算的重平衡", and
+ *     "5 Fun Projects for LLM Inference Engineering", section 2: attention is
+ *     computed tile by tile with a running max and running sum (online softmax),
+ *     never materialising the full score matrix; the result is exact attention.
+ *
+ * Layouts (all row-major, bf16 = IEEE bfloat16):
+ *   k_cache, v_cache : [NB][Hkv][bs][D]   one (block, kv head) page is contiguous
+ *   block_tables     : [B][MB] int32      physical block of logical page p of
+ *                                          sequence b; entries past the last
+ *                                          used page are never read
+ *   context_lens     : [B] int32          number of valid keys of sequence b,
+ *                                          including rows just written
+ *   slot_mapping     : [T] int64          slot = block * bs + offset; < 0 = skip
+ *   Grouped-query heads: query head h reads kv head h / (Hq / Hkv).
+ *
+ * Conventions:
+ *   - Ownership: the caller owns every buffer (device memory unless stated).
+ *     The library allocates no device memory; it keeps one static device error
+ *     word per device.  Workspace for the split-KV path is passed in.
+ *   - Asynchrony: every call only enqueues kernels on `stream` and returns;
+ *     nothing synchronises except pkv_get_device_error.
+ *   - Errors: argument checks happen on the host before any launch and return
+ *     a status without launching.  A failed launch returns PKV_ERR_CUDA.
+ *     Problems only the device can see (a slot or block id outside the pool, a
+ *     context length larger than the block table, a wait that ran out) set
+ *     the device error word, read with pkv_get_device_error.
+ *   - Supported now: dtype PKV_BF16; decode and prefill need bs = 16 and
+ *     D in {64, 128} (decode) or D = 128 (prefill); the cache write takes any
+ *     bs and any D that is a multiple of 8.  All pointers 16-byte aligned.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pkv_status {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer      */
+  PKV_ERR_UNSUPPORTED = 2,  /* valid but not built: dtype, D, bs, group size   */
+  PKV_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed            */
+  PKV_ERR_TIMEOUT = 4,      /* device: a bounded wait gave up                  */
+  PKV_ERR_BOUNDS = 5,       /* device: slot / block id / length out of range   */
+  PKV_ERR_WORKSPACE = 6     /* workspace missing or smaller than required      */
+} pkv_status;
+
+typedef enum pkv_dtype { PKV_BF16 = 0 } pkv_dtype;
+
+/* A cudaStream_t (NULL = the legacy default stream). */
+typedef void* pkv_stream_t;
+
+/*
+ * kv_cache_write -- scatter new K/V rows into their physical slots.
+ * For every token t with s = slot_mapping[t] >= 0 and every kv head h:
+ *   k_cache[s / bs][h][s % bs][:] = key[t][h][:]   (and the same for V).
+ * A bit copy: the result is exact.  Tiny-Infer page, section
+ * "分页KV缓存：借鉴操作系统的内存管理" (logical position -> physical block).
+ *   key, value       : device, [T][Hkv][D] bf16; token stride in ELEMENTS
+ *                      (>= Hkv*D, a multiple of 8), head stride D
+ *   k_cache, v_cache : device, [NB][Hkv][bs][D] bf16, written in place
+ *   slot_mapping     : device, [T] int64; < 0 skips the token; >= NB*bs sets
+ *                      PKV_ERR_BOUNDS on the device and skips the token
+ * T = 0 launches nothing.  Returns PKV_ERR_INVALID_ARG for null pointers,
+ * negative sizes or misalignment, PKV_ERR_UNSUPPORTED for D % 8 != 0.
+ */
+pkv_status pkv_kv_cache_write(const void* key, const void* value,
+                              int64_t key_stride_tok, int64_t value_stride_tok,
+                              void* k_cache, void* v_cache,
+                              const int64_t* slot_mapping, int32_t T,
+                              int32_t Hkv, int32_t D, int32_t NB, int32_t bs,
+                              pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * paged_attention -- decode: one query token per sequence against its paged
+ * K/V, grouped-query heads, online softmax in one pass over the pages.
+ *   out[b][h][:] = sum_j softmax_j(scale * q[b][h] . k_j) v_j over the
+ *   context_lens[b] keys of sequence b (0 keys -> a zero row).
+ *   out          : device, [B][Hq][D] bf16
+ *   q            : device, [B][Hq][D] bf16
+ *   block_tables : device, [B][MB] int32; context_lens: device, [B] int32
+ *   max_context_len_hint : host upper bound on context_lens (<= 0: MB*bs);
+ *                  used only to size the launch, never checked against the
+ *                  device values, which are never read on the host
+ *   workspace    : device scratch for split-KV partials, or NULL.  With at
+ *                  least pkv_paged_attention_workspace_size(...) bytes the
+ *                  call may split long contexts across CTAs and merge the
+ *                  parts by log-sum-exp; with less it runs one CTA per
+ *                  (sequence, head group) and needs none.
+ * Same shape limits as the file header; Hq % Hkv == 0.
+ */
+pkv_status pkv_paged_attention(void* out, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* block_tables,
+                               int32_t MB, const int32_t* context_lens,
+                               int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                               int32_t NB, int32_t bs, float scale,
+                               int32_t max_context_len_hint, void* workspace,
+                               size_t workspace_bytes, pkv_dtype dtype,
+                               pkv_stream_t stream);
+
+/* Workspace bytes pkv_paged_attention may use for these sizes on the current
+ * device (0 if it would never split). */
+size_t pkv_paged_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv,
+                                          int32_t D, int32_t MB, int32_t bs,
+                                          int32_t max_context_len_hint);
+
+/*
+ * paged_attention_split -- the split-KV ("flash-decoding") path with an
+ * explicit split size.  Split c of sequence b covers logical pages
+ * [c*pages_per_split, (c+1)*pages_per_split); each CTA writes its normalised
+ * partial o_c and its log-sum-exp, and a second kernel merges
+ *   out = sum_c e^{lse_c - M} o_c / sum_c e^{lse_c - M},  M = max_c lse_c.
+ * Same result as pkv_paged_attention up to rounding.  The split-KV form is
+ * not on the pages; it answers their remark that variable-length batches need
+ * padding or bucketing ("Triton融合算子优化：LLM推理性能提升3倍的工程实践",
+ * section 六).  pages_per_split >= 1; num_splits = ceil(ceil(max_ctx/bs) /
+ * pages_per_split) where max_ctx = max_context_len_hint (<= 0: MB*bs); the
+ * device sets PKV_ERR_BOUNDS if a context is longer than that.
+ *   workspace: device, >= pkv_split_workspace_size(B, Hq, D, num_splits) bytes.
+ */
+pkv_status pkv_paged_attention_split(void* out, const void* q,
+                                     const void* k_cache, const void* v_cache,
+                                     const int32_t* block_tables, int32_t MB,
+                                     const int32_t* context_lens, int32_t B,
+                                     int32_t Hq, int32_t Hkv, int32_t D,
+                                     int32_t NB, int32_t bs, float scale,
+                                     int32_t max_context_len_hint,
+                                     int32_t pages_per_split, void* workspace,
+                                     size_t workspace_bytes, pkv_dtype dtype,
+                                     pkv_stream_t stream);
+
+/* Workspace bytes of the split path: fp32 partials [B][Hq][C][D] plus fp32
+ * log-sum-exp [B][Hq][C], each 256-byte aligned. */
+size_t pkv_split_workspace_size(int32_t B, int32_t Hq, int32_t D,
+                                int32_t num_splits);
+
+/*
+ * paged_attention_prefill -- causal chunked prefill over the paged cache.
+ * Sequence b has a chunk of Q_b = query_start_loc[b+1] - query_start_loc[b]
+ * new queries, which are the LAST Q_b of its context_lens[b] positions; their
+ * K/V must already be in the cache (written by pkv_kv_cache_write).  Query i
+ * sits at position L_b - Q_b + i and attends to keys 0 .. L_b - Q_b + i.
+ * Runs on the tcgen05 tensor cores with TMEM accumulators: S = Q K^T and
+ * O += P V are bf16 MMAs with fp32 accumulation, P rounded to bf16.
+ * Tiny-Infer page, sections "Flash Attention：内存与计算的重平衡" and
+ * "分页KV缓存：借鉴操作系统的内存管理".
+ *   out             : device, [sumQ][Hq][D] bf16
+ *   q               : device, [sumQ][Hq][D] bf16
+ *   query_start_loc : device, [B+1] int32, query_start_loc[0] = 0
+ *   max_q_len       : host upper bound on Q_b (sizes the launch)
+ * Needs D = 128, bs = 16, Hq / Hkv dividing 128.
+ */
+pkv_status pkv_paged_attention_prefill(
+    void* out, const void* q, const int32_t* query_start_loc,
+    const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    int32_t MB, const int32_t* context_lens, int32_t B, int32_t sumQ,
+    int32_t max_q_len, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+    int32_t bs, float scale, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error
+ * word (0 = none, else a pkv_status value recorded by a kernel).
+ */
+pkv_status pkv_get_device_error(pkv_stream_t stream, int32_t* err_out);
+
+/* Number of kernels the last successful call on this host thread launched. */
+int32_t pkv_last_launch_count(void);
+
+/* Static text for a status code. */
+const char* pkv_status_string(pkv_status status);
+
+/*
+ * Self-test of the bounded waits: launches one CTA that waits on a barrier
+ * nothing will complete, with a limit of timeout_us microseconds; the kernel
+ * then records PKV_ERR_TIMEOUT in the device error word and returns, leaving
+ * the context usable.  For tests of the failure path; hangs nothing.
+ */
+pkv_status pkv_selftest_wait_timeout(uint32_t timeout_us, pkv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

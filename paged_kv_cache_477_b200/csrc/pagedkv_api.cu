@@ -1,0 +1,382 @@
+// pagedkv_api.cu -- the extern "C" boundary of libpagedkv.so.
+//
+// Host side only: validate arguments, pick a launch shape from host-known
+// sizes (never from device data), enqueue kernels on the caller's stream.
+// See include/pagedkv.h for the contract of every entry point.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "decode_attn.cuh"
+#include "kv_cache_write.cuh"
+#include "pkv_common.cuh"
+
+namespace {
+
+thread_local int32_t t_launches = 0;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+pkv_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+int device_sm_count(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+    cache[dev] = sms;
+  }
+  return cache[dev];
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ----------------------------------------------------------------- decode --
+constexpr int kDecodeWarps = 4;
+constexpr int stages_for(int D) { return D == 128 ? 8 : 16; }  // 64 KB ring either way
+
+template <int D, int HG>
+using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D)>;
+
+template <int D, int HG>
+struct DecodeKernel {
+  static constexpr auto fn = pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D)>;
+  // set the dynamic shared-memory limit once per device; return CTAs per SM
+  static int prepare(int dev) {
+    static int occ[kMaxDevices] = {0};
+    static std::mutex mu;
+    if (dev < 0 || dev >= kMaxDevices) return 1;
+    std::lock_guard<std::mutex> g(mu);
+    if (occ[dev] == 0) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess)
+        return -1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DecodeS<D, HG>::THREADS,
+                                                        DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess ||
+          n <= 0)
+        return -1;
+      occ[dev] = n;
+    }
+    return occ[dev];
+  }
+};
+
+int heads_per_cta(int G) {
+  if (G % 4 == 0) return 4;
+  if (G % 2 == 0) return 2;
+  return 1;
+}
+
+int decode_occupancy(int D, int HG, int dev) {
+  if (D == 128) {
+    if (HG == 4) return DecodeKernel<128, 4>::prepare(dev);
+    if (HG == 2) return DecodeKernel<128, 2>::prepare(dev);
+    return DecodeKernel<128, 1>::prepare(dev);
+  }
+  if (HG == 4) return DecodeKernel<64, 4>::prepare(dev);
+  if (HG == 2) return DecodeKernel<64, 2>::prepare(dev);
+  return DecodeKernel<64, 1>::prepare(dev);
+}
+
+struct DecodePlan {
+  int num_splits;
+  int pages_per_split;
+  size_t workspace;
+};
+
+int max_pages_of(int32_t MB, int32_t bs, int32_t hint) {
+  const int64_t cap = (int64_t)MB * bs;
+  const int64_t ctx = (hint > 0) ? std::min<int64_t>(hint, cap) : cap;
+  return (int)((ctx + pkv::kPageRows - 1) / pkv::kPageRows);
+}
+
+size_t split_ws_bytes(int32_t B, int32_t Hq, int32_t D, int32_t C) {
+  const size_t rows = (size_t)B * Hq * C;
+  return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
+}
+
+// Host-only choice of the split count.  Aim for at least four waves of CTAs
+// so the block scheduler can balance ragged lengths, but keep every split at
+// least kMinSplitPages pages long so per-CTA set-up stays amortised.
+constexpr int kMinSplitPages = 32;
+constexpr int kTargetWaves = 4;
+
+DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, int32_t bs,
+                     int32_t hint) {
+  DecodePlan pl{1, std::max<int32_t>(MB, 1), 0};
+  const int max_pages = max_pages_of(MB, bs, hint);
+  const int G = Hq / Hkv, HG = heads_per_cta(G);
+  const int64_t units = (int64_t)B * Hkv * (G / HG);
+  const int dev = current_device();
+  const int occ = std::max(1, decode_occupancy(D, HG, dev));
+  const int64_t slots = (int64_t)device_sm_count(dev) * occ;
+  if (units <= 0 || max_pages <= kMinSplitPages) return pl;
+  int64_t C = (kTargetWaves * slots + units - 1) / units;
+  C = std::min<int64_t>(C, max_pages / kMinSplitPages);
+  if (C <= 1) return pl;
+  const int pps = (int)((max_pages + C - 1) / C);
+  pl.pages_per_split = pps;
+  pl.num_splits = (max_pages + pps - 1) / pps;
+  pl.workspace = split_ws_bytes(B, Hq, D, pl.num_splits);
+  return pl;
+}
+
+template <int D, int HG>
+pkv_status launch_decode_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C,
+                           cudaStream_t st) {
+  if (DecodeKernel<D, HG>::prepare(current_device()) < 0) return PKV_ERR_CUDA;
+  dim3 grid(C, Hkv * nsub, B);
+  DecodeKernel<D, HG>::fn<<<grid, DecodeS<D, HG>::THREADS, DecodeS<D, HG>::SMEM_BYTES, st>>>(p);
+  return launch_status();
+}
+
+template <int D>
+pkv_status launch_merge_t(const pkv::MergeParams& mp, int B, int Hq, cudaStream_t st) {
+  pkv::lse_merge_kernel<D><<<dim3(Hq, B), D, 0, st>>>(mp);
+  return launch_status();
+}
+
+pkv_status check_decode_args(void* out, const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, int32_t MB, const int32_t* context_lens,
+                             int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB, int32_t bs,
+                             pkv_dtype dtype) {
+  if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || NB < 0 || MB < 0 || bs <= 0) return PKV_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return PKV_ERR_UNSUPPORTED;
+  if (bs != pkv::kPageRows) return PKV_ERR_UNSUPPORTED;
+  if (B == 0) return PKV_OK;
+  if (!out || !q || !context_lens || ((MB > 0) && (!block_tables || !k_cache || !v_cache)))
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_ERR_INVALID_ARG;
+  return PKV_OK;
+}
+
+pkv_status run_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                      const int32_t* block_tables, int32_t MB, const int32_t* context_lens,
+                      int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB, float scale,
+                      const DecodePlan& pl, void* workspace, cudaStream_t st) {
+  const int G = Hq / Hkv, HG = heads_per_cta(G), nsub = G / HG;
+  const int C = pl.num_splits;
+  pkv::DecodeParams p{};
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_cache = static_cast<const unsigned char*>(k_cache);
+  p.v_cache = static_cast<const unsigned char*>(v_cache);
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NB = NB; p.MB = MB;
+  p.G = G; p.nsub = nsub;
+  p.pages_per_split = pl.pages_per_split;
+  p.num_splits = C;
+  p.cap_tokens = (int32_t)std::min<int64_t>((int64_t)MB, (int64_t)C * pl.pages_per_split) * pkv::kPageRows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (C > 1) {
+    const size_t rows = (size_t)B * Hq * C;
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) +
+                                          round256(rows * D * sizeof(float)));
+  }
+  pkv_status s;
+  if (D == 128)
+    s = HG == 4 ? launch_decode_t<128, 4>(p, B, Hkv, nsub, C, st)
+        : HG == 2 ? launch_decode_t<128, 2>(p, B, Hkv, nsub, C, st)
+                  : launch_decode_t<128, 1>(p, B, Hkv, nsub, C, st);
+  else
+    s = HG == 4 ? launch_decode_t<64, 4>(p, B, Hkv, nsub, C, st)
+        : HG == 2 ? launch_decode_t<64, 2>(p, B, Hkv, nsub, C, st)
+                  : launch_decode_t<64, 1>(p, B, Hkv, nsub, C, st);
+  if (s != PKV_OK) return s;
+  int launches = 1;
+  if (C > 1) {
+    pkv::MergeParams mp{};
+    mp.out = p.out;
+    mp.o_part = p.o_part;
+    mp.lse_part = p.lse_part;
+    mp.context_lens = context_lens;
+    mp.Hq = Hq;
+    mp.num_splits = C;
+    mp.pages_per_split = pl.pages_per_split;
+    mp.cap_tokens = p.cap_tokens;
+    s = D == 128 ? launch_merge_t<128>(mp, B, Hq, st) : launch_merge_t<64>(mp, B, Hq, st);
+    if (s != PKV_OK) return s;
+    ++launches;
+  }
+  t_launches = launches;
+  return PKV_OK;
+}
+
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    pkv::mbar_init(pkv::smem_addr(&bar), 1);
+    pkv::fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on this barrier: the bounded wait must give up,
+  // record PKV_ERR_TIMEOUT and return.
+  if (threadIdx.x == 0) pkv::mbar_wait(pkv::smem_addr(&bar), 0, limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status s) {
+  switch (s) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID_ARG: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PKV_ERR_CUDA: return "CUDA error";
+    case PKV_ERR_TIMEOUT: return "device wait timed out";
+    case PKV_ERR_BOUNDS: return "index out of range on the device";
+    case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int32_t pkv_last_launch_count(void) { return t_launches; }
+
+pkv_status pkv_kv_cache_write(const void* key, const void* value, int64_t key_stride_tok,
+                              int64_t value_stride_tok, void* k_cache, void* v_cache,
+                              const int64_t* slot_mapping, int32_t T, int32_t Hkv, int32_t D,
+                              int32_t NB, int32_t bs, pkv_dtype dtype, pkv_stream_t stream) {
+  t_launches = 0;
+  if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (T < 0 || Hkv <= 0 || D <= 0 || NB < 0 || bs <= 0) return PKV_ERR_INVALID_ARG;
+  if (D % 8 != 0) return PKV_ERR_UNSUPPORTED;
+  if (T == 0) return PKV_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_ERR_INVALID_ARG;
+  if (key_stride_tok < (int64_t)Hkv * D || value_stride_tok < (int64_t)Hkv * D ||
+      key_stride_tok % 8 != 0 || value_stride_tok % 8 != 0)
+    return PKV_ERR_INVALID_ARG;
+  pkv::KvWriteParams p{};
+  p.key = static_cast<const uint4*>(key);
+  p.value = static_cast<const uint4*>(value);
+  p.key_stride_vec = key_stride_tok / 8;
+  p.value_stride_vec = value_stride_tok / 8;
+  p.k_cache = static_cast<uint4*>(k_cache);
+  p.v_cache = static_cast<uint4*>(v_cache);
+  p.slot_mapping = slot_mapping;
+  p.vec_per_row = D / 8;
+  p.total_vec = (int64_t)T * Hkv * p.vec_per_row;
+  p.pool_slots = (int64_t)NB * bs;
+  p.Hkv = Hkv;
+  p.bs = bs;
+  const int threads = 256;
+  const int64_t blocks = (p.total_vec + threads - 1) / threads;
+  if (blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
+  pkv::kv_cache_write_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  pkv_status s = launch_status();
+  if (s == PKV_OK) t_launches = 1;
+  return s;
+}
+
+size_t pkv_split_workspace_size(int32_t B, int32_t Hq, int32_t D, int32_t num_splits) {
+  if (B <= 0 || Hq <= 0 || D <= 0 || num_splits <= 1) return 0;
+  return split_ws_bytes(B, Hq, D, num_splits);
+}
+
+size_t pkv_paged_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t D,
+                                          int32_t MB, int32_t bs, int32_t max_context_len_hint) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || (D != 64 && D != 128) || bs != pkv::kPageRows)
+    return 0;
+  return plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint).workspace;
+}
+
+pkv_status pkv_paged_attention(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* block_tables, int32_t MB,
+                               const int32_t* context_lens, int32_t B, int32_t Hq, int32_t Hkv,
+                               int32_t D, int32_t NB, int32_t bs, float scale,
+                               int32_t max_context_len_hint, void* workspace,
+                               size_t workspace_bytes, pkv_dtype dtype, pkv_stream_t stream) {
+  t_launches = 0;
+  pkv_status s = check_decode_args(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq,
+                                    Hkv, D, NB, bs, dtype);
+  if (s != PKV_OK || B == 0) return s;
+  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint);
+  if (pl.num_splits > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned16(workspace)))
+    pl = DecodePlan{1, std::max<int32_t>(MB, 1), 0};  // no room: one CTA per head group
+  if (pl.num_splits == 1) pl.pages_per_split = std::max<int32_t>(MB, 1);
+  return run_decode(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq, Hkv, D, NB,
+                    scale, pl, workspace, static_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_paged_attention_split(void* out, const void* q, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables, int32_t MB,
+                                     const int32_t* context_lens, int32_t B, int32_t Hq,
+                                     int32_t Hkv, int32_t D, int32_t NB, int32_t bs, float scale,
+                                     int32_t max_context_len_hint, int32_t pages_per_split,
+                                     void* workspace, size_t workspace_bytes, pkv_dtype dtype,
+                                     pkv_stream_t stream) {
+  t_launches = 0;
+  pkv_status s = check_decode_args(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq,
+                                    Hkv, D, NB, bs, dtype);
+  if (s != PKV_OK) return s;
+  if (pages_per_split <= 0) return PKV_ERR_INVALID_ARG;
+  if (B == 0) return PKV_OK;
+  const int max_pages = std::max(1, max_pages_of(MB, bs, max_context_len_hint));
+  DecodePlan pl{(max_pages + pages_per_split - 1) / pages_per_split, pages_per_split, 0};
+  if (pl.num_splits > 1) {
+    pl.workspace = split_ws_bytes(B, Hq, D, pl.num_splits);
+    if (!workspace || workspace_bytes < pl.workspace || !aligned16(workspace))
+      return PKV_ERR_WORKSPACE;
+  }
+  return run_decode(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq, Hkv, D, NB,
+                    scale, pl, workspace, static_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* query_start_loc,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, int32_t MB,
+                                       const int32_t* context_lens, int32_t B, int32_t sumQ,
+                                       int32_t max_q_len, int32_t Hq, int32_t Hkv, int32_t D,
+                                       int32_t NB, int32_t bs, float scale, pkv_dtype dtype,
+                                       pkv_stream_t stream) {
+  t_launches = 0;
+  (void)out; (void)q; (void)query_start_loc; (void)k_cache; (void)v_cache; (void)block_tables;
+  (void)MB; (void)context_lens; (void)B; (void)sumQ; (void)max_q_len; (void)Hq; (void)Hkv;
+  (void)D; (void)NB; (void)bs; (void)scale; (void)dtype; (void)stream;
+  return PKV_ERR_UNSUPPORTED;
+}
+
+pkv_status pkv_get_device_error(pkv_stream_t stream, int32_t* err_out) {
+  if (!err_out) return PKV_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return PKV_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, pkv::g_error_word, sizeof(int)) != cudaSuccess) return PKV_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(pkv::g_error_word, &zero, sizeof(int)) != cudaSuccess) return PKV_ERR_CUDA;
+  *err_out = v;
+  return PKV_OK;
+}
+
+pkv_status pkv_selftest_wait_timeout(uint32_t timeout_us, pkv_stream_t stream) {
+  t_launches = 0;
+  if (timeout_us == 0 || timeout_us > 5000000u) return PKV_ERR_INVALID_ARG;
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      (uint64_t)timeout_us * 1000ull);
+  pkv_status s = launch_status();
+  if (s == PKV_OK) t_launches = 1;
+  return s;
+}
+
+}  // extern "C"

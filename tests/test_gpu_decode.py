@@ -1,0 +1,208 @@
+"""GPU parity of the cache write and decode attention against the fp64 oracle.
+
+Every call goes through the C ABI (via the ctypes binding).  Cache writes must
+be bit-exact over the whole pool; attention must satisfy
+|gpu - ref| <= 5e-3 + 1e-2 |ref| element by element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_477_b200 as pkv
+from paged_kv_cache_477_b200 import workloads as wl
+from paged_kv_cache_477_b200.workloads import bf16_bits
+from parity import HostCase, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from paged_kv_cache_477_b200 import build
+    build.build()
+    pkv.load_library()
+    pkv.get_device_error()  # start from a clean error word
+    yield
+
+
+def _no_device_error():
+    assert pkv.get_device_error() == 0
+
+
+# --------------------------------------------------------------------------- #
+# kv_cache_write                                                               #
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("T,Hkv,D,bs,NB", [(37, 2, 64, 16, 9), (128, 8, 128, 16, 64), (5, 3, 8, 4, 4),
+                                         (300, 1, 256, 8, 50)])
+def test_kv_cache_write_bit_exact(T, Hkv, D, bs, NB):
+    g = torch.Generator(device="cuda").manual_seed(T * 7 + D)
+    k_cache = torch.randn(NB, Hkv, bs, D, device="cuda", generator=g).to(torch.bfloat16)
+    v_cache = torch.randn(NB, Hkv, bs, D, device="cuda", generator=g).to(torch.bfloat16)
+    key = torch.randn(T, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
+    val = torch.randn(T, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
+    gc = torch.Generator().manual_seed(T)
+    slots = torch.randperm(NB * bs, generator=gc)[:T].to(torch.int64)
+    slots[::7] = -1                                     # padding tokens are skipped
+    k_host, v_host = bf16_bits(k_cache).copy(), bf16_bits(v_cache).copy()
+    oracle.get().kv_cache_write(bf16_bits(key), bf16_bits(val), k_host, v_host, slots.numpy())
+    pkv.kv_cache_write(key, val, k_cache, v_cache, slots.cuda())
+    assert pkv.last_launch_count() == 1
+    assert np.array_equal(bf16_bits(k_cache), k_host)
+    assert np.array_equal(bf16_bits(v_cache), v_host)
+    _no_device_error()
+
+
+def test_kv_cache_write_strided_rows():
+    """key/value taken as column slices of a fused [T, 3*Hkv*D] projection."""
+    T, Hkv, D, bs, NB = 20, 2, 64, 16, 4
+    g = torch.Generator(device="cuda").manual_seed(3)
+    qkv = torch.randn(T, 3 * Hkv * D, device="cuda", generator=g).to(torch.bfloat16)
+    key = qkv[:, Hkv * D:2 * Hkv * D].view(T, Hkv, D)
+    val = qkv[:, 2 * Hkv * D:].view(T, Hkv, D)
+    k_cache = torch.zeros(NB, Hkv, bs, D, device="cuda", dtype=torch.bfloat16)
+    v_cache = torch.zeros_like(k_cache)
+    slots = torch.arange(T, dtype=torch.int64, device="cuda") * 3 % (NB * bs)
+    k_host, v_host = bf16_bits(k_cache).copy(), bf16_bits(v_cache).copy()
+    oracle.get().kv_cache_write(bf16_bits(key.contiguous()), bf16_bits(val.contiguous()), k_host, v_host,
+                                slots.cpu().numpy())
+    pkv.kv_cache_write(key, val, k_cache, v_cache, slots)
+    assert np.array_equal(bf16_bits(k_cache), k_host)
+    assert np.array_equal(bf16_bits(v_cache), v_host)
+    _no_device_error()
+
+
+def test_kv_cache_write_out_of_range_slot_is_reported_and_skipped():
+    NB, Hkv, bs, D = 2, 1, 16, 64
+    k_cache = torch.zeros(NB, Hkv, bs, D, device="cuda", dtype=torch.bfloat16)
+    v_cache = torch.zeros_like(k_cache)
+    key = torch.ones(2, Hkv, D, device="cuda", dtype=torch.bfloat16)
+    slots = torch.tensor([NB * bs, 5], dtype=torch.int64, device="cuda")
+    pkv.kv_cache_write(key, key, k_cache, v_cache, slots)
+    assert pkv.get_device_error() == 5
+    assert float(k_cache.float().sum()) == D            # only slot 5 was written
+
+
+def test_kv_cache_write_empty_is_noop():
+    k_cache = torch.zeros(1, 1, 16, 64, device="cuda", dtype=torch.bfloat16)
+    e = torch.empty(0, 1, 64, device="cuda", dtype=torch.bfloat16)
+    pkv.kv_cache_write(e, e, k_cache, k_cache, torch.empty(0, dtype=torch.int64, device="cuda"))
+    assert pkv.last_launch_count() == 0
+
+
+# --------------------------------------------------------------------------- #
+# decode                                                                       #
+# --------------------------------------------------------------------------- #
+
+def _decode_case(lens, Hq, Hkv, D, seed, write_tokens=0, pool_extra=3):
+    pages = sum(-(-L // 16) for L in lens)
+    return wl.make_case(B=len(lens), Hq=Hq, Hkv=Hkv, D=D, bs=16, lens=lens, seed=seed, device="cuda",
+                        pool_blocks=pages + pool_extra, write_tokens=write_tokens)
+
+
+def test_decode_tiny_workload():
+    case = wl.workload("tiny_decode", device="cuda")
+    host = HostCase(case)
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale)
+    assert_close(out, host.decode_ref(), "tiny_decode")
+    _no_device_error()
+
+
+EDGE_LENS = [0, 1, 15, 16, 17, 31, 32, 33, 100, 257, 600]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2), (8, 2), (16, 2), (6, 2), (32, 8)])
+def test_decode_shapes_and_edges(D, Hq, Hkv):
+    case = _decode_case(EDGE_LENS, Hq, Hkv, D, seed=100 + D + Hq)
+    host = HostCase(case)
+    ref = host.decode_ref()
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale)
+    assert_close(out, ref, f"auto D={D} G={Hq // Hkv}")
+    assert torch.count_nonzero(out[0]) == 0              # empty context -> zero row
+    for pps in (1, 2, 3, 7):
+        out_s = pkv.paged_attention_split(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                          case.context_lens, case.scale, pages_per_split=pps)
+        assert_close(out_s, ref, f"split pps={pps} D={D} G={Hq // Hkv}")
+    _no_device_error()
+
+
+def test_decode_llama32_1b_workload_full():
+    case = wl.workload("llama32_1b_decode", device="cuda")
+    host = HostCase(case)
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale, max_context_len=4096)
+    assert_close(out, host.decode_ref(), "llama32_1b_decode")
+    _no_device_error()
+
+
+def test_decode_llama3_8b_workload_with_write_sampled():
+    """The bench's launch sequence: cache write of one token per sequence, then decode."""
+    case = wl.workload("llama3_8b_decode", device="cuda")
+    host = HostCase(case)                       # pre-write pool, copied before any kernel runs
+    pkv.kv_cache_write(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping)
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale, max_context_len=4096)
+    host.apply_write()
+    # the write is bit-exact over the whole pool
+    assert np.array_equal(bf16_bits(case.k_cache), host.k)
+    assert np.array_equal(bf16_bits(case.v_cache), host.v)
+    rows = [0, 1, 37, 64, 101, 127]
+    assert_close(out[rows], host.decode_ref(rows), "llama3_8b_decode sampled")
+    _no_device_error()
+
+
+def test_decode_ragged_long_workload_sampled():
+    case = wl.workload("ragged_long_decode", device="cuda")
+    host = HostCase(case)
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale, max_context_len=32768)
+    assert pkv.last_launch_count() == 2               # split-KV partials + merge
+    lens = np.array(case.lens)
+    long_rows = list(np.where(lens == 32768)[0][:2])
+    short_rows = list(np.argsort(lens)[:4])
+    rows = long_rows + short_rows
+    assert_close(out[rows], host.decode_ref(rows), "ragged_long_decode sampled")
+    _no_device_error()
+
+
+def test_split_count_invariance():
+    case = _decode_case([2000, 37, 900, 1], 8, 2, 128, seed=9)
+    ref = HostCase(case).decode_ref()
+    outs = []
+    for pps in (1, 4, 16, 64, 1000):
+        outs.append(pkv.paged_attention_split(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                              case.context_lens, case.scale, pages_per_split=pps))
+        assert_close(outs[-1], ref, f"pps={pps}")
+    for o in outs[1:]:
+        d = (o.float() - outs[0].float()).abs().max().item()
+        assert d <= 2 * (5e-3 + 1e-2 * outs[0].float().abs().max().item())
+
+
+def test_decode_bad_block_id_is_reported():
+    case = _decode_case([40, 40], 4, 2, 64, seed=5)
+    bt = case.block_tables.clone()
+    bt[1, 1] = case.NB + 5                            # outside the pool
+    pkv.paged_attention(case.q, case.k_cache, case.v_cache, bt, case.context_lens, case.scale)
+    assert pkv.get_device_error() == 5
+
+
+def test_decode_context_longer_than_table_is_reported():
+    case = _decode_case([40], 4, 2, 64, seed=6)
+    lens = torch.tensor([40 + 16 * 8], dtype=torch.int32, device="cuda")
+    pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, lens, case.scale)
+    assert pkv.get_device_error() == 5
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    pkv.selftest_wait_timeout(2000)                   # 2 ms limit on a barrier nobody completes
+    assert pkv.get_device_error() == 4
+    case = wl.workload("tiny_decode", device="cuda")
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale)
+    assert_close(out, HostCase(case).decode_ref(), "after timeout")
+    _no_device_error()
