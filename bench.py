@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
+    ap.add_argument("--profile", default=None, choices=["decode", "split", "prefill", "write"],
+                    help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
 
@@ -290,8 +292,43 @@ def extras(peaks):
 # --------------------------------------------------------------------------- #
 # main arm                                                                     #
 # --------------------------------------------------------------------------- #
+def profile_case(kind: str, launches: int = 3):
+    """A few launches of one kernel on a case small enough for a full ncu
+    capture (a few GB on the device at most, inputs still larger than L2)."""
+    import paged_kv_cache_477_b200 as pkv
+    from paged_kv_cache_477_b200 import workloads as wl
+    torch.cuda.set_device(0)
+    if kind in ("decode", "split", "write"):
+        # 32 of the Llama-3-8B-shaped sequences: 512 MiB of K/V
+        c = wl.make_case(B=32, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 32, seed=1003, device="cuda",
+                         write_tokens=1)
+        out = torch.empty_like(c.q)
+        for _ in range(launches):
+            if kind == "write":
+                pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)
+            elif kind == "decode":
+                pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale,
+                                    out=out, max_context_len=4096)
+            else:
+                pkv.paged_attention_split(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens,
+                                          c.scale, pages_per_split=32, out=out, max_context_len=4096)
+    else:
+        c = wl.workload("chunked_prefill", device="cuda")
+        pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)
+        out = torch.empty_like(c.q)
+        for _ in range(launches):
+            pkv.paged_attention_prefill(c.q, c.query_start_loc, c.k_cache, c.v_cache, c.block_tables,
+                                        c.context_lens, c.scale, c.max_q_len, out=out)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+    print(f"profile case {kind}: ok")
+
+
 def main():
     args = parse()
+    if args.profile:
+        profile_case(args.profile)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -13,16 +13,22 @@
 //   * One CTA = (sequence b, a group of HG query heads sharing one kv head,
 //     a range of pages).  The HG query rows live in registers, so every K/V
 //     byte is read from HBM once per group (grouped-query reuse).
-//   * Warp NW is the producer: one lane issues 1-D bulk copies (cp.async.bulk)
+//   * Every warp feeds itself: lane 0 issues 1-D bulk copies (cp.async.bulk)
 //     of whole pages -- a (block, kv head) page is one contiguous 4 KB (D=128)
-//     or 2 KB (D=64) run -- into a STAGES-deep shared-memory ring, completion
-//     tracked by mbarriers.  Block-table entries are fetched 32 at a time.
-//   * Warps 0..NW-1 consume pages round-robin.  A key row is split over
-//     LPR = D/16 lanes (16 elements, two 16-byte vectors each), so a warp
-//     covers 32/LPR rows per instruction and a dot product needs only
-//     log2(LPR) shuffle steps.  Each lane keeps its own running max, sum and
-//     fp32 accumulator for the rows it sees; warps and lanes merge once at the
-//     end by log-sum-exp.
+//     or 2 KB (D=64) run -- into the warp's own SW-stage shared-memory ring,
+//     completion tracked by one mbarrier per stage.  A warp refills a stage
+//     as soon as it has read it, so no cross-warp hand-off is needed and no
+//     warp is spent on copies.  Block-table entries are fetched 32 at a time,
+//     one chunk ahead.
+//   * Two CTAs per SM (shared-memory carveout at its maximum) keep
+//     2 x NW x SW pages -- about 192 KB -- in flight per SM, which is what
+//     Little's law asks for at full HBM bandwidth.
+//   * A key row is split over LPR = D/16 lanes (16 elements, two 16-byte
+//     vectors each), so a warp covers 32/LPR rows per instruction and a dot
+//     product needs only log2(LPR) shuffle steps.  Products and P.V updates
+//     use packed fp32 (FFMA2) on element pairs.  Each lane keeps its own
+//     running max, sum and fp32 accumulator; lanes and warps merge once at
+//     the end by log-sum-exp.
 //   * Split mode (num_splits > 1): each CTA writes its normalised partial and
 //     its log2-domain log-sum-exp; lse_merge_kernel combines them.
 //   * Shared-memory reads are conflict-free: for D=128 the 8 lanes of a row
@@ -54,7 +60,7 @@ struct DecodeParams {
   float scale_log2;              // scale * log2(e)
 };
 
-template <int D, int HG, int NW, int STAGES>
+template <int D, int HG, int NW, int SW>
 struct DecodeShape {
   static_assert(D == 64 || D == 128, "head_dim");
   static constexpr int LPR = D / 16;              // lanes sharing one key row
@@ -62,17 +68,24 @@ struct DecodeShape {
   static constexpr int TPL = kPageRows / RPW;     // rows per lane per page
   static constexpr int PAGE_BYTES = kPageRows * D * 2;
   static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;  // K page + V page
-  static constexpr int THREADS = (NW + 1) * 32;
-  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
-  static constexpr int MERGE_FLOATS = NW * HG * D + 2 * NW * HG;
-  static constexpr int BAR_OFFSET = RING_BYTES + MERGE_FLOATS * 4;
-  static constexpr int SMEM_BYTES = BAR_OFFSET + 2 * STAGES * 8;
+  static constexpr int THREADS = NW * 32;
+  static constexpr int WARP_RING = SW * STAGE_BYTES;
+  static constexpr int RING_BYTES = NW * WARP_RING;
+  // after its last page a warp reuses its own ring for the merge data
+  static constexpr int MERGE_BYTES = (HG * D + 2 * HG) * 4;
+  static_assert(MERGE_BYTES <= WARP_RING, "merge data must fit the warp's ring");
+  static constexpr int BAR_OFFSET = RING_BYTES;
+  static constexpr int SMEM_BYTES = BAR_OFFSET + NW * SW * 8;
 };
 
-template <int D, int HG, int NW, int STAGES>
-__global__ void __launch_bounds__((NW + 1) * 32)
+__device__ __forceinline__ float2 widen2(uint32_t w) {
+  return make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
+}
+
+template <int D, int HG, int NW, int SW>
+__global__ void __launch_bounds__(NW * 32)
     decode_attn_kernel(const __grid_constant__ DecodeParams p) {
-  using S = DecodeShape<D, HG, NW, STAGES>;
+  using S = DecodeShape<D, HG, NW, SW>;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int split = blockIdx.x, hsub = blockIdx.y, b = blockIdx.z;
@@ -104,117 +117,106 @@ __global__ void __launch_bounds__((NW + 1) * 32)
     return;
   }
 
-  const uint32_t ring = smem_addr(smem);
-  const uint32_t bars = ring + S::BAR_OFFSET;
-  auto full = [&](int s) { return bars + 8u * s; };
-  auto empty = [&](int s) { return bars + 8u * (STAGES + s); };
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full(s), 1);
-      mbar_init(empty(s), 1);
-    }
+  // ------------------------------------------------ this warp's page stream --
+  const int my_n = warp < n ? (n - warp + NW - 1) / NW : 0;  // pages warp, warp+NW, ...
+  const uint32_t wring = smem_addr(smem) + warp * S::WARP_RING;
+  const uint32_t wbar = smem_addr(smem) + S::BAR_OFFSET + warp * SW * 8;
+  unsigned char* wring_ptr = smem + warp * S::WARP_RING;
+  if (lane == 0) {
+    for (int s = 0; s < SW; ++s) mbar_init(wbar + 8 * s, 1);
     fence_barrier_init();
   }
-  __syncthreads();
+  __syncwarp();
 
-  if (warp == NW) {
-    // ------------------------------------------------------------ producer --
-    const int32_t* bt = p.block_tables + (size_t)b * p.MB + pg0;
-    const uint64_t pol = policy_evict_first();  // every page is read once
-    int issued = 0;
-    bool ok = true;
-    for (int i0 = 0; i0 < n && ok; i0 += 32) {
-      int blk = 0;
-      if (i0 + lane < n) {
-        blk = __ldg(bt + i0 + lane);
-        if (blk < 0 || blk >= p.NB) {
-          set_error(PKV_ERR_BOUNDS);
-          blk = 0;  // keep every copy inside the pool
-        }
-      }
-      const int cnt = min(32, n - i0);
-      for (int j = 0; j < cnt; ++j) {
-        const int bj = __shfl_sync(0xffffffffu, blk, j);
-        const int i = i0 + j, s = i % STAGES;
-        if (lane == 0) {
-          if (i >= STAGES) ok = mbar_wait(empty(s), ((i / STAGES) & 1) ^ 1);
-          if (ok) {
-            const size_t off = ((size_t)bj * p.Hkv + kvh) * S::PAGE_BYTES;
-            mbar_arrive_expect_tx(full(s), S::STAGE_BYTES);
-            bulk_g2s_hint(ring + s * S::STAGE_BYTES, p.k_cache + off, S::PAGE_BYTES, full(s), pol);
-            bulk_g2s_hint(ring + s * S::STAGE_BYTES + S::PAGE_BYTES, p.v_cache + off,
-                          S::PAGE_BYTES, full(s), pol);
-            ++issued;
-          }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+  const int32_t* btw = p.block_tables + (size_t)b * p.MB + pg0 + warp;  // entry of page j: btw[j*NW]
+  auto load_chunk = [&](int c) {
+    const int j = c * 32 + lane;
+    int blk = 0;
+    if (j < my_n) {
+      blk = __ldg(btw + (size_t)j * NW);
+      if (blk < 0 || blk >= p.NB) {
+        set_error(PKV_ERR_BOUNDS);
+        blk = 0;  // keep every copy inside the pool
       }
     }
-    // Do not leave while a copy into this CTA's shared memory may be in
-    // flight: wait for the last issued use of every stage to land.
+    return blk;
+  };
+  int bt_cur = load_chunk(0), bt_nxt = load_chunk(1), chunk = 0;
+  const uint64_t pol = policy_evict_first();  // every page is read once
+  int issued = 0;
+  auto issue_next = [&]() {  // warp-uniform; pages are issued in order
+    const int k = issued;
+    if ((k >> 5) != chunk) {
+      bt_cur = bt_nxt;
+      chunk = k >> 5;
+      bt_nxt = load_chunk(chunk + 1);
+    }
+    const int blk = __shfl_sync(0xffffffffu, bt_cur, k & 31);
     if (lane == 0) {
-      for (int s = 0; s < STAGES && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / STAGES) * STAGES;
-        mbar_wait(full(s), (last / STAGES) & 1);
-      }
+      const int s = k % SW;
+      const size_t off = ((size_t)blk * p.Hkv + kvh) * S::PAGE_BYTES;
+      mbar_arrive_expect_tx(wbar + 8 * s, S::STAGE_BYTES);
+      bulk_g2s_hint(wring + s * S::STAGE_BYTES, p.k_cache + off, S::PAGE_BYTES, wbar + 8 * s, pol);
+      bulk_g2s_hint(wring + s * S::STAGE_BYTES + S::PAGE_BYTES, p.v_cache + off, S::PAGE_BYTES,
+                    wbar + 8 * s, pol);
     }
-    return;
-  }
+    ++issued;
+  };
+  for (int k = 0; k < SW && k < my_n; ++k) issue_next();
 
-  // -------------------------------------------------------------- consumers --
+  // ---------------------------------------------------------- registers --
   const int rg = lane / S::LPR, sub = lane % S::LPR;
   const int swap = (D == 64) ? (rg & 1) : 0;
   const int ch0 = sub + S::LPR * swap;        // 16-byte vector held in slot 0
   const int ch1 = sub + S::LPR * (swap ^ 1);  // and in slot 1
 
-  float qf[HG][16];
+  float2 q2[HG][8];  // the lane's 16 q elements as 8 pairs, pre-scaled
 #pragma unroll
   for (int h = 0; h < HG; ++h) {
     const uint4* qrow = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + head0 + h) * D);
-    widen8(__ldg(qrow + ch0), qf[h]);
-    widen8(__ldg(qrow + ch1), qf[h] + 8);
+    const uint4 a = __ldg(qrow + ch0), c = __ldg(qrow + ch1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) qf[h][e] *= p.scale_log2;
+    for (int e = 0; e < 8; ++e) q2[h][e] = __fmul2_rn(widen2(w[e]), sc2);
   }
 
-  float m[HG], l[HG], acc[HG][16];
+  float m[HG], l[HG];
+  float2 acc2[HG][8];
 #pragma unroll
   for (int h = 0; h < HG; ++h) {
     m[h] = -INFINITY;
     l[h] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) acc[h][e] = 0.f;
+    for (int e = 0; e < 8; ++e) acc2[h][e] = make_float2(0.f, 0.f);
   }
 
   const int L_local = L - pg0 * kPageRows;  // valid rows counted from this CTA's first page
-  for (int i = warp; i < n; i += NW) {
-    const int s = i % STAGES;
+  int done = 0;
+  for (int j = 0; j < my_n; ++j, ++done) {
+    const int s = j % SW;
     // every lane waits (each needs the acquire); a timeout on any lane stops
-    // the whole warp, which still joins the merge below
-    const bool ok = mbar_wait(full(s), (i / STAGES) & 1);
+    // the whole warp, which still drains its copies and joins the merge
+    const bool ok = mbar_wait(wbar + 8 * s, (j / SW) & 1);
     if (!__all_sync(0xffffffffu, ok)) break;
-    const unsigned char* kp = smem + s * S::STAGE_BYTES;
+    const unsigned char* kp = wring_ptr + s * S::STAGE_BYTES;
     const unsigned char* vp = kp + S::PAGE_BYTES;
-    const int row0 = i * kPageRows;
+    const int row0 = (warp + j * NW) * kPageRows;
 
     float sc[S::TPL][HG];
 #pragma unroll
     for (int t = 0; t < S::TPL; ++t) {
       const int r = rg + t * S::RPW;
       const uint4* krow = reinterpret_cast<const uint4*>(kp + r * D * 2);
-      float kf[16];
-      widen8(krow[ch0], kf);
-      widen8(krow[ch1], kf + 8);
+      const uint4 ka = krow[ch0], kb = krow[ch1];
+      const float2 k2[8] = {widen2(ka.x), widen2(ka.y), widen2(ka.z), widen2(ka.w),
+                            widen2(kb.x), widen2(kb.y), widen2(kb.z), widen2(kb.w)};
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
-        float d0 = 0.f, d1 = 0.f;
+        float2 d = __fmul2_rn(q2[h][0], k2[0]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          d0 = fmaf(qf[h][e], kf[e], d0);
-          d1 = fmaf(qf[h][8 + e], kf[8 + e], d1);
-        }
-        sc[t][h] = d0 + d1;
+        for (int e = 1; e < 8; ++e) d = __ffma2_rn(q2[h][e], k2[e], d);
+        sc[t][h] = d.x + d.y;
       }
     }
 #pragma unroll
@@ -245,8 +247,9 @@ __global__ void __launch_bounds__((NW + 1) * 32)
         const float alpha = (mn == -INFINITY) ? 1.f : ex2(m[h] - mn);
         m[h] = mn;
         l[h] *= alpha;
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[h][e] *= alpha;
+        for (int e = 0; e < 8; ++e) acc2[h][e] = __fmul2_rn(acc2[h][e], a2);
       }
     }
 #pragma unroll
@@ -254,25 +257,41 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       if (!valid[t]) continue;  // canary / stale rows are never touched
       const int r = rg + t * S::RPW;
       const uint4* vrow = reinterpret_cast<const uint4*>(vp + r * D * 2);
-      float vf[16];
-      widen8(vrow[ch0], vf);
-      widen8(vrow[ch1], vf + 8);
+      const uint4 va = vrow[ch0], vb = vrow[ch1];
+      const float2 v2[8] = {widen2(va.x), widen2(va.y), widen2(va.z), widen2(va.w),
+                            widen2(vb.x), widen2(vb.y), widen2(vb.z), widen2(vb.w)};
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
         const float pr = ex2(sc[t][h] - m[h]);
         l[h] += pr;
+        const float2 pp = make_float2(pr, pr);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[h][e] = fmaf(pr, vf[e], acc[h][e]);
+        for (int e = 0; e < 8; ++e) acc2[h][e] = __ffma2_rn(pp, v2[e], acc2[h][e]);
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty(s));
+    if (issued < my_n) {
+      // the stage just read is refilled: order the generic-proxy reads of all
+      // lanes before the copy engine's writes
+      fence_proxy_async_smem();
+      __syncwarp();
+      issue_next();
+    }
   }
+  // Never reuse or leave the ring while one of this warp's copies may still
+  // land in it (only possible after a timeout): wait for the last issued use
+  // of every stage.
+  if (done < issued && lane == 0) {
+    for (int s = 0; s < SW && s < issued; ++s) {
+      const int last = s + ((issued - 1 - s) / SW) * SW;
+      mbar_wait(wbar + 8 * s, (last / SW) & 1);
+    }
+  }
+  __syncwarp();
 
   // ---- merge the row groups of this warp (lanes with the same D-slice) ----
 #pragma unroll
   for (int off = S::LPR; off < 32; off <<= 1) {
-    const int flip = (D == 64 && off == S::LPR) ? 8 : 0;  // partner keeps the other order
+    const int flip = (D == 64 && off == S::LPR) ? 4 : 0;  // partner keeps the other order
 #pragma unroll
     for (int h = 0; h < HG; ++h) {
       const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
@@ -280,48 +299,54 @@ __global__ void __launch_bounds__((NW + 1) * 32)
       const float mn = fmaxf(m[h], mo);
       const float a = (mn == -INFINITY) ? 0.f : ex2(m[h] - mn);
       const float c = (mn == -INFINITY) ? 0.f : ex2(mo - mn);
-      float recv[16];
+      float2 recv[8];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) recv[e] = __shfl_xor_sync(0xffffffffu, acc[h][e ^ flip], off);
+      for (int e = 0; e < 8; ++e) {
+        recv[e].x = __shfl_xor_sync(0xffffffffu, acc2[h][e ^ flip].x, off);
+        recv[e].y = __shfl_xor_sync(0xffffffffu, acc2[h][e ^ flip].y, off);
+      }
+      const float2 a2 = make_float2(a, a), c2 = make_float2(c, c);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) acc[h][e] = acc[h][e] * a + recv[e] * c;
+      for (int e = 0; e < 8; ++e) acc2[h][e] = __ffma2_rn(acc2[h][e], a2, __fmul2_rn(recv[e], c2));
       l[h] = l[h] * a + lo * c;
       m[h] = mn;
     }
   }
 
-  // ---- merge the warps through shared memory -------------------------------
-  float* sm_acc = reinterpret_cast<float*>(smem + S::RING_BYTES);  // [NW][HG][D]
-  float* sm_m = sm_acc + NW * HG * D;                               // [NW][HG]
-  float* sm_l = sm_m + NW * HG;
-  if (rg == 0) {  // lanes 0..LPR-1 hold the warp's result in natural order
+  // ---- merge the warps through shared memory (each warp's own ring) -------
+  {
+    float* mine = reinterpret_cast<float*>(wring_ptr);  // [HG][D] acc, [HG] m, [HG] l
+    if (rg == 0) {  // lanes 0..LPR-1 hold the warp's result in natural order
 #pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      float4* dst = reinterpret_cast<float4*>(sm_acc + (warp * HG + h) * D);
-      dst[2 * ch0] = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-      dst[2 * ch0 + 1] = make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
-      dst[2 * ch1] = make_float4(acc[h][8], acc[h][9], acc[h][10], acc[h][11]);
-      dst[2 * ch1 + 1] = make_float4(acc[h][12], acc[h][13], acc[h][14], acc[h][15]);
-      if (sub == 0) {
-        sm_m[warp * HG + h] = m[h];
-        sm_l[warp * HG + h] = l[h];
+      for (int h = 0; h < HG; ++h) {
+        float4* dst = reinterpret_cast<float4*>(mine + h * D);
+        dst[2 * ch0] = make_float4(acc2[h][0].x, acc2[h][0].y, acc2[h][1].x, acc2[h][1].y);
+        dst[2 * ch0 + 1] = make_float4(acc2[h][2].x, acc2[h][2].y, acc2[h][3].x, acc2[h][3].y);
+        dst[2 * ch1] = make_float4(acc2[h][4].x, acc2[h][4].y, acc2[h][5].x, acc2[h][5].y);
+        dst[2 * ch1 + 1] = make_float4(acc2[h][6].x, acc2[h][6].y, acc2[h][7].x, acc2[h][7].y);
+        if (sub == 0) {
+          mine[HG * D + h] = m[h];
+          mine[HG * D + HG + h] = l[h];
+        }
       }
     }
   }
-  named_barrier_sync(1, NW * 32);
+  __syncthreads();
   for (int idx = threadIdx.x; idx < HG * D; idx += NW * 32) {
     const int h = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w * HG + h]);
+    for (int w = 0; w < NW; ++w)
+      M = fmaxf(M, reinterpret_cast<const float*>(smem + w * S::WARP_RING)[HG * D + h]);
     float Ls = 0.f, A = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const float mw = sm_m[w * HG + h];
+      const float* part = reinterpret_cast<const float*>(smem + w * S::WARP_RING);
+      const float mw = part[HG * D + h];
       if (mw == -INFINITY) continue;  // this warp saw no valid row
       const float wt = ex2(mw - M);
-      Ls = fmaf(sm_l[w * HG + h], wt, Ls);
-      A = fmaf(sm_acc[(w * HG + h) * D + d], wt, A);
+      Ls = fmaf(part[HG * D + HG + h], wt, Ls);
+      A = fmaf(part[h * D + d], wt, A);
     }
     const size_t row = (size_t)b * p.Hq + head0 + h;
     if (p.num_splits == 1) {

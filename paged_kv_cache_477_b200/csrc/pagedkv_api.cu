@@ -47,7 +47,9 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ----------------------------------------------------------------- decode --
 constexpr int kDecodeWarps = 4;
-constexpr int stages_for(int D) { return D == 128 ? 8 : 16; }  // 64 KB ring either way
+// stages per warp: 3 x 8 KB (D=128) or 6 x 4 KB (D=64) -> 96 KB of pages in
+// flight per CTA, two CTAs per SM
+constexpr int stages_for(int D) { return D == 128 ? 3 : 6; }
 
 template <int D, int HG>
 using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D)>;
@@ -63,7 +65,9 @@ struct DecodeKernel {
     std::lock_guard<std::mutex> g(mu);
     if (occ[dev] == 0) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess)
+                               DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return -1;
       int n = 0;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DecodeS<D, HG>::THREADS,
