@@ -25,7 +25,9 @@
  * Conventions:
  *   - Ownership: the caller owns every buffer (device memory unless stated).
  *     The library allocates no device memory; it keeps one static device error
- *     word per device.  Workspace for the split-KV path is passed in.
+ *     word per device, and the static scratch array of
+ *     pkv_paged_attention_split_noalloc.  Workspace for the split-KV path is
+ *     otherwise passed in.
  *   - Asynchrony: every call only enqueues kernels on `stream` and returns;
  *     nothing synchronises except pkv_get_device_error.
  *   - Errors: argument checks happen on the host before any launch and return
@@ -145,6 +147,38 @@ pkv_status pkv_paged_attention_split(void* out, const void* q,
  * log-sum-exp [B][Hq][C], each 256-byte aligned. */
 size_t pkv_split_workspace_size(int32_t B, int32_t Hq, int32_t D,
                                 int32_t num_splits);
+
+/*
+ * paged_attention_split_noalloc -- pkv_paged_attention_split for callers that
+ * cannot allocate device memory: an engine plugin whose enqueue hook must not
+ * allocate, a serving loop that cannot take the device-wide synchronisation a
+ * cudaMalloc may cause, or a process whose device memory is already reserved
+ * in full by another allocator.  The pages have no counterpart of this call;
+ * it exists for those callers only.
+ *   Same arguments and result as pkv_paged_attention_split without the
+ *   workspace: the split partials go to one static device array of
+ *   PKV_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads
+ *   it, until the process exits.  The caller still owns out and every input.
+ *   - A request whose partials need more than PKV_NOALLOC_SCRATCH_BYTES
+ *     (pkv_split_workspace_size(B, Hq, D, num_splits)) returns
+ *     PKV_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Nothing is allocated or freed by this call, by the library or through
+ *     any library routine.
+ *   - Every call shares the one array and leaves its partials in it; every
+ *     partial the merge reads is written first by the same call, so nothing
+ *     needs clearing.  Calls that overlap on the GPU (other streams, other
+ *     host threads) race on the array: serialise them.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (8u << 20) /* 8 MiB per GPU */
+
+pkv_status pkv_paged_attention_split_noalloc(
+    void* out, const void* q, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, int32_t MB, const int32_t* context_lens,
+    int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB, int32_t bs,
+    float scale, int32_t max_context_len_hint, int32_t pages_per_split,
+    pkv_dtype dtype, pkv_stream_t stream);
 
 /*
  * paged_attention_prefill -- causal chunked prefill over the paged cache.

@@ -46,6 +46,8 @@ EXPORTS = {
     "pkv_paged_attention_split": ([_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32,
                                    _F32, _I32, _I32, _P, _SZ, _I32, _P], _I32),
     "pkv_split_workspace_size": ([_I32, _I32, _I32, _I32], _SZ),
+    "pkv_paged_attention_split_noalloc": ([_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
+                                           _I32, _F32, _I32, _I32, _I32, _P], _I32),
     "pkv_paged_attention_prefill": ([_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                      _I32, _I32, _I32, _F32, _I32, _P], _I32),
     "pkv_get_device_error": ([_P, ctypes.POINTER(_I32)], _I32),
@@ -207,6 +209,28 @@ def paged_attention_split(q, k_cache, v_cache, block_tables, context_lens, scale
                                        int(max_context_len), int(pages_per_split), ws_ptr, ws_bytes,
                                        PKV_BF16, _stream(stream))
     _check(rc, "paged_attention_split")
+    return out
+
+
+# Bytes of the library's static split-KV scratch (one array per GPU).
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def paged_attention_split_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                                  pages_per_split: int, out=None, max_context_len: int = 0,
+                                  stream=None) -> torch.Tensor:
+    """Split-KV decode for callers that must not allocate device memory.
+
+    Same result as paged_attention_split, but the split partials live in a
+    static array inside the library (NOALLOC_SCRATCH_BYTES per GPU), so the
+    call allocates nothing.  Pass ``out`` to keep this wrapper allocation-free
+    as well.  Calls that overlap on the GPU share that array and race."""
+    NB, Hkv, bs, D, B, Hq, MB, out = _decode_common(q, k_cache, v_cache, block_tables, context_lens, out)
+    rc = load_library().pkv_paged_attention_split_noalloc(
+        out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_tables.data_ptr(), MB,
+        context_lens.data_ptr(), B, Hq, Hkv, D, NB, bs, float(scale), int(max_context_len),
+        int(pages_per_split), PKV_BF16, _stream(stream))
+    _check(rc, "paged_attention_split_noalloc")
     return out
 
 

@@ -384,3 +384,60 @@ pkv_status pkv_selftest_wait_timeout(uint32_t timeout_us, pkv_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Split-KV decode without any allocation by the caller.
+//
+// Some callers cannot hand the library a workspace: engine plugins whose
+// enqueue hook must not allocate, serving loops that cannot afford the device
+// synchronisation a cudaMalloc may cause, or processes whose device memory is
+// already reserved in full by another allocator.  For them the split-KV
+// partials live in this file-scope device array instead.  It is created when
+// the library's device code is loaded on a GPU and stays there until the
+// process exits (PKV_NOALLOC_SCRATCH_BYTES on every GPU that loads it).
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+// Host code cannot use g_noalloc_scratch's name as a device address: on the
+// host it only stands in for the symbol.  Its device address is looked up once
+// per device, with that device current, and kept here.
+void* noalloc_scratch_address(int dev) {
+  static void* addr[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> g(mu);
+  if (addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return nullptr;
+    addr[dev] = ptr;
+  }
+  return addr[dev];
+}
+
+}  // namespace
+
+extern "C" pkv_status pkv_paged_attention_split_noalloc(
+    void* out, const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    int32_t MB, const int32_t* context_lens, int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+    int32_t bs, float scale, int32_t max_context_len_hint, int32_t pages_per_split, pkv_dtype dtype,
+    pkv_stream_t stream) {
+  t_launches = 0;
+  pkv_status s = check_decode_args(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq,
+                                    Hkv, D, NB, bs, dtype);
+  if (s != PKV_OK) return s;
+  if (pages_per_split <= 0) return PKV_ERR_INVALID_ARG;
+  if (B == 0) return PKV_OK;
+  const int max_pages = std::max(1, max_pages_of(MB, bs, max_context_len_hint));
+  DecodePlan pl{(max_pages + pages_per_split - 1) / pages_per_split, pages_per_split, 0};
+  void* scratch = nullptr;
+  if (pl.num_splits > 1) {
+    pl.workspace = split_ws_bytes(B, Hq, D, pl.num_splits);
+    if (pl.workspace > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_WORKSPACE;
+    scratch = noalloc_scratch_address(current_device());
+    if (scratch == nullptr) return PKV_ERR_CUDA;
+  }
+  return run_decode(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq, Hkv, D, NB,
+                    scale, pl, scratch, static_cast<cudaStream_t>(stream));
+}
