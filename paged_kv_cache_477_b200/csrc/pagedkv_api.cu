@@ -9,9 +9,12 @@
 #include <cstdint>
 #include <mutex>
 
+#include <cuda.h>
+
 #include "decode_attn.cuh"
 #include "kv_cache_write.cuh"
 #include "pkv_common.cuh"
+#include "prefill_attn.cuh"
 
 namespace {
 
@@ -226,6 +229,51 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   return PKV_OK;
 }
 
+// ---------------------------------------------------------------- prefill --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map with a 128-byte swizzle; dims/box innermost first, strides
+// in bytes for dims 1..rank-1.
+bool make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+               const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+             strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int prefill_prepare(int dev) {
+  static int done[kMaxDevices] = {0};
+  static std::mutex mu;
+  if (dev < 0 || dev >= kMaxDevices) return -1;
+  std::lock_guard<std::mutex> g(mu);
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(pkv::prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pkv::pf::SMEM_BYTES) != cudaSuccess)
+      return -1;
+    done[dev] = 1;
+  }
+  return 0;
+}
+
 __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -356,10 +404,51 @@ pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* 
                                        int32_t NB, int32_t bs, float scale, pkv_dtype dtype,
                                        pkv_stream_t stream) {
   t_launches = 0;
-  (void)out; (void)q; (void)query_start_loc; (void)k_cache; (void)v_cache; (void)block_tables;
-  (void)MB; (void)context_lens; (void)B; (void)sumQ; (void)max_q_len; (void)Hq; (void)Hkv;
-  (void)D; (void)NB; (void)bs; (void)scale; (void)dtype; (void)stream;
-  return PKV_ERR_UNSUPPORTED;
+  if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (B < 0 || sumQ < 0 || max_q_len < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || NB < 0 || MB < 0 || bs <= 0)
+    return PKV_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (D != pkv::pf::D || bs != pkv::kPageRows || G > pkv::pf::BM || pkv::pf::BM % G != 0)
+    return PKV_ERR_UNSUPPORTED;
+  if (!(scale >= 0.f) || scale == INFINITY) return PKV_ERR_UNSUPPORTED;  // also rejects NaN
+  if (B == 0 || sumQ == 0 || max_q_len == 0) return PKV_OK;
+  if (!out || !q || !query_start_loc || !k_cache || !v_cache || !block_tables || !context_lens ||
+      NB == 0 || MB == 0)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
+    return PKV_ERR_INVALID_ARG;
+  const int dev = current_device();
+  if (prefill_prepare(dev) < 0) return PKV_ERR_CUDA;
+
+  CUtensorMap tm_q, tm_k, tm_v;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)sumQ};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)(pkv::pf::BM / G)};
+    if (!make_tmap(&tm_q, q, 3, dims, strides, box)) return PKV_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)bs, (cuuint64_t)Hkv, (cuuint64_t)NB};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)bs * D * 2, (cuuint64_t)Hkv * bs * D * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)bs, 1, 1};
+    if (!make_tmap(&tm_k, k_cache, 4, dims, strides, box)) return PKV_ERR_CUDA;
+    if (!make_tmap(&tm_v, v_cache, 4, dims, strides, box)) return PKV_ERR_CUDA;
+  }
+  pkv::PrefillParams p{};
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.query_start_loc = query_start_loc;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NB = NB; p.MB = MB; p.G = G; p.sumQ = sumQ;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int ppt = pkv::pf::BM / G;
+  dim3 grid((max_q_len + ppt - 1) / ppt, Hkv, B);
+  pkv::prefill_attn_kernel<<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
+      p, tm_q, tm_k, tm_v);
+  pkv_status s = launch_status();
+  if (s == PKV_OK) t_launches = 1;
+  return s;
 }
 
 pkv_status pkv_get_device_error(pkv_stream_t stream, int32_t* err_out) {

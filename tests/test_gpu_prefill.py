@@ -1,0 +1,109 @@
+"""GPU parity of the tcgen05 chunked causal prefill against the fp64 oracle.
+
+The chunk's K/V rows are written by the library's cache write first, as a
+caller would; the oracle applies its own cache write to the generator's
+pre-write pool.  Attention outputs must satisfy |gpu - ref| <= 5e-3 + 1e-2 |ref|.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_477_b200 as pkv
+from paged_kv_cache_477_b200 import workloads as wl
+from parity import HostCase, assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from paged_kv_cache_477_b200 import build
+    build.build()
+    pkv.load_library()
+    pkv.get_device_error()
+    yield
+
+
+def _run(case):
+    host = HostCase(case)
+    pkv.kv_cache_write(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping)
+    out = pkv.paged_attention_prefill(case.q, case.query_start_loc, case.k_cache, case.v_cache,
+                                      case.block_tables, case.context_lens, case.scale, case.max_q_len)
+    assert pkv.last_launch_count() == 1
+    host.apply_write()
+    return out, host
+
+
+def _prefill_case(lens, qlens, Hq, Hkv, seed, extra_blocks=2):
+    pages = sum(-(-L // 16) for L in lens)
+    return wl.make_case(kind="prefill", B=len(lens), Hq=Hq, Hkv=Hkv, D=128, bs=16, lens=lens, q_len=qlens,
+                        seed=seed, device="cuda", pool_blocks=pages + extra_blocks)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (32, 8), (4, 4), (16, 8), (16, 2)])
+def test_prefill_small_full(Hq, Hkv):
+    # ragged chunks, partial last pages (NaN canaries in the tails), a chunk that
+    # is the whole context, single-token chunks, several Q tiles per sequence
+    lens = [200, 77, 300, 1, 129, 45]
+    qlens = [130, 77, 33, 1, 1, 45]
+    case = _prefill_case(lens, qlens, Hq, Hkv, seed=500 + Hq + Hkv)
+    out, host = _run(case)
+    ref, tok = host.prefill_ref()
+    assert_close(out[tok], ref, f"prefill Hq={Hq} Hkv={Hkv}")
+    assert pkv.get_device_error() == 0
+
+
+def test_prefill_empty_chunk_and_long_chunk():
+    lens = [16, 700, 64]
+    qlens = [0, 700, 2]          # a sequence with nothing new, a 700-token chunk, a short one
+    case = _prefill_case(lens, qlens, 32, 8, seed=600)
+    out, host = _run(case)
+    ref, tok = host.prefill_ref()
+    assert_close(out[tok], ref, "prefill empty/long chunk")
+    assert pkv.get_device_error() == 0
+
+
+def test_prefill_workload_sampled_rows():
+    """The bench's prefill workload (B=4, 512-token chunks after 3584 cached
+    tokens).  Sampled rows: each is checked against decode attention over the
+    keys its position may see, which the oracle's causal pin ties to the
+    chunked definition."""
+    case = wl.workload("chunked_prefill", device="cuda")
+    out, host = _run(case)
+    qsl = host.qsl
+    rows, qs_rows, lens = [], [], []
+    for b in range(case.B):
+        Q, L = int(qsl[b + 1] - qsl[b]), int(host.lens[b])
+        for i in (0, 1, 31, 32, 127, 128, 255, 300, 510, Q - 1):
+            rows.append(b)
+            qs_rows.append(int(qsl[b]) + i)
+            lens.append(L - Q + i + 1)
+    ref = oracle.get().paged_attention(np.ascontiguousarray(host.q[qs_rows]), host.k, host.v,
+                                       np.ascontiguousarray(host.bt[rows]), np.array(lens, np.int32),
+                                       case.scale)
+    assert_close(out[qs_rows], ref, "chunked_prefill sampled rows")
+    assert pkv.get_device_error() == 0
+
+
+def test_prefill_matches_decode_on_last_row():
+    """The last query of a chunk is a decode step over the whole context."""
+    case = _prefill_case([513, 1000], [100, 513], 32, 8, seed=601)
+    out, host = _run(case)
+    qsl = host.qsl
+    last = [int(qsl[1]) - 1, int(qsl[2]) - 1]
+    q_dec = case.q[last].contiguous()
+    dec = pkv.paged_attention(q_dec, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale)
+    d = (out[last].float() - dec.float()).abs().max().item()
+    assert d <= 2e-2, d
+
+
+def test_prefill_rejects_unsupported_shapes():
+    case = _prefill_case([32], [16], 8, 2, seed=602)
+    with pytest.raises(pkv.PagedKVError) as e:
+        pkv.paged_attention_prefill(case.q, case.query_start_loc, case.k_cache, case.v_cache,
+                                    case.block_tables, case.context_lens, -1.0, case.max_q_len)
+    assert e.value.status == 2
+    assert pkv.last_launch_count() == 0
