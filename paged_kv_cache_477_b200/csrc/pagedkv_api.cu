@@ -269,6 +269,11 @@ int prefill_prepare(int dev) {
     if (cudaFuncSetAttribute(pkv::prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pkv::pf::SMEM_BYTES) != cudaSuccess)
       return -1;
+    // the kernel's setmaxnreg split is sized for exactly this register count
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, pkv::prefill_attn_kernel) != cudaSuccess ||
+        attr.numRegs != pkv::pf::REGS_LAUNCH)
+      return -2;
     done[dev] = 1;
   }
   return 0;
@@ -419,7 +424,9 @@ pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* 
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
   const int dev = current_device();
-  if (prefill_prepare(dev) < 0) return PKV_ERR_CUDA;
+  const int prep = prefill_prepare(dev);
+  if (prep == -2) return PKV_ERR_UNSUPPORTED;  // build with an unexpected register count
+  if (prep < 0) return PKV_ERR_CUDA;
 
   CUtensorMap tm_q, tm_k, tm_v;
   {
@@ -442,8 +449,8 @@ pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* 
   p.context_lens = context_lens;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NB = NB; p.MB = MB; p.G = G; p.sumQ = sumQ;
   p.scale_log2 = scale * 1.4426950408889634f;
-  const int ppt = pkv::pf::BM / G;
-  dim3 grid((max_q_len + ppt - 1) / ppt, Hkv, B);
+  const int ppc = pkv::pf::NQT * (pkv::pf::BM / G);  // query positions per CTA
+  dim3 grid((max_q_len + ppc - 1) / ppc, Hkv, B);
   pkv::prefill_attn_kernel<<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
       p, tm_q, tm_k, tm_v);
   pkv_status s = launch_status();
