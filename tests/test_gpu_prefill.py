@@ -107,3 +107,12 @@ def test_prefill_rejects_unsupported_shapes():
                                     case.block_tables, case.context_lens, -1.0, case.max_q_len)
     assert e.value.status == 2
     assert pkv.last_launch_count() == 0
+
+
+def test_prefill_zero_scale_gives_mean_of_visible_values():
+    case = wl.make_case(kind="prefill", B=2, Hq=8, Hkv=2, D=128, bs=16, lens=[150, 40], q_len=[70, 40],
+                        seed=603, device="cuda", scale=0.0)
+    out, host = _run(case)
+    ref, tok = host.prefill_ref()
+    assert_close(out[tok], ref, "prefill scale=0")
+    assert pkv.get_device_error() == 0
