@@ -41,12 +41,15 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          out: str | None = None) -> str:
+    """Compile the library (to ``out``, default the in-tree libpagedkv.so)."""
+    target = out or LIB
+    if not force and out is None and up_to_date():
         return LIB
     cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
            "-shared", "-Xcompiler", "-fPIC,-O2", "-I", os.path.join(ROOT, "include"),
-           "-o", LIB + ".tmp", SRC]
+           "-o", target + ".tmp", SRC]
     if verbose:
         cmd += ["-Xptxas", "-v"]
     if extra:
@@ -56,8 +59,8 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         print(res.stdout + res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(target + ".tmp", target)
+    return target
 
 
 if __name__ == "__main__":

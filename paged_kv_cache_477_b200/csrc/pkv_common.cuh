@@ -11,7 +11,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/pagedkv.h"
+#include "pagedkv.h"  // from include/ (nvcc -I include)
 
 #ifndef PKV_WAIT_LIMIT_NS
 #define PKV_WAIT_LIMIT_NS 1000000000ull  // 1 s: far above any legitimate wait

@@ -83,12 +83,23 @@ constexpr int TMEM_COLS = 512;
 constexpr int TILE_COLS = 256;  // query tile i: scores at i*256, O at i*256 + 128
 constexpr int O_COL = 128;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
-constexpr int POLY_PAIR_EVERY = 4;  // one column pair in four takes the FMA-pipe exp2
+#ifndef PKV_PREFILL_POLY_EVERY
+#define PKV_PREFILL_POLY_EVERY 0  // measured fastest on B200: MUFU for every exponential
+#endif
+// one column pair in POLY_PAIR_EVERY takes the FMA-pipe exp2 (0: none)
+constexpr int POLY_PAIR_EVERY = PKV_PREFILL_POLY_EVERY;
 constexpr int REGS_LAUNCH = 168;    // 65536 / 384 rounded down to a multiple of 8
-constexpr int REGS_LOW = 56;        // load / MMA / allocator warpgroup
-constexpr int REGS_HIGH = 224;      // softmax warpgroups
+constexpr int REGS_LOW = 64;        // load / MMA / allocator warpgroup
+constexpr int REGS_HIGH = 216;      // softmax warpgroups
 static_assert(4 * REGS_LOW + 8 * REGS_HIGH <= 12 * REGS_LAUNCH, "register split must fit the launch");
 }  // namespace pf
+
+// Three-input maximum (one ALU instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
 // 2^x on the FMA pipe (Cody-Waite style): x = n + f with n = round(x) found by
 // the 1.5 * 2^23 shifter, f in [-0.5, 0.5]; 2^f by a degree-3 polynomial
@@ -255,16 +266,21 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       const int tail_rows = L % 16;
       const int tail_page = (L - 1) / 16;
 
+      // Descriptors are built once; a K step only moves the start address,
+      // whose 14-bit field (address >> 4) cannot carry: shared memory < 256 KB.
+      const uint64_t desc_q = tc::smem_desc_sw128(base + pf::Q_OFF, 16, 1024);
+      const uint64_t desc_k = tc::smem_desc_sw128(base + pf::K_OFF, 16, 1024);
+      const uint64_t desc_v = tc::smem_desc_sw128(base + pf::V_OFF, pf::HALF_BYTES, 1024);
+      constexpr uint32_t TILE16 = pf::TILE_BYTES >> 4;
       auto qk = [&](int i, int j) {  // S_i = Q_i K_j^T
         const int ks = j % pf::KSTAGES;
         if (lane == 0) {
-          const uint32_t q_s = base + pf::Q_OFF + i * pf::TILE_BYTES;
-          const uint32_t k_s = base + pf::K_OFF + ks * pf::TILE_BYTES;
-  #pragma unroll
+          const uint64_t dq = desc_q + i * TILE16, dk = desc_k + ks * TILE16;
+          const uint32_t d_s = tmem + i * pf::TILE_COLS;
+#pragma unroll
           for (int kk = 0; kk < pf::D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * pf::HALF_BYTES + (kk & 3) * 32;
-            tc::mma_ss(tmem + i * pf::TILE_COLS, tc::smem_desc_sw128(q_s + off, 16, 1024),
-                       tc::smem_desc_sw128(k_s + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+            const uint32_t off16 = ((kk >> 2) * pf::HALF_BYTES + (kk & 3) * 32) >> 4;
+            tc::mma_ss(d_s, dq + off16, dk + off16, IDESC_S, kk > 0 ? 1u : 0u);
           }
           tc::commit(bar(pf::B_SFULL + i));
           if (i == pf::NQT - 1) tc::commit(bar(pf::B_KEMPTY + ks));
@@ -292,13 +308,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         }
         tc::fence_after_sync();
         if (lane == 0) {
-          const uint32_t v_s = base + pf::V_OFF + vs * pf::TILE_BYTES;
+          const uint64_t dv = desc_v + vs * TILE16;
           const uint32_t p_t = tmem + i * pf::TILE_COLS;
-  #pragma unroll
+          const uint32_t d_o = p_t + pf::O_COL;
+#pragma unroll
           for (int kk = 0; kk < pf::BN / 16; ++kk)
-            tc::mma_ts(tmem + i * pf::TILE_COLS + pf::O_COL, p_t + kk * 8,
-                       tc::smem_desc_sw128(v_s + kk * 2048, pf::HALF_BYTES, 1024), IDESC_PV,
-                       (t > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_ts(d_o, p_t + kk * 8, dv + kk * (2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
           tc::commit(bar(pf::B_OREADY + i));
           if (i == pf::NQT - 1) tc::commit(bar(pf::B_VEMPTY + vs));
         }
@@ -363,13 +378,18 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         for (int c = 0; c < pf::BN; ++c)
           if (kv0 + c > limit) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx0 = __uint_as_float(sr[0]), mx1 = __uint_as_float(sr[1]);
+      // row max: eight independent chains of three-input maxima
+      float mxk[8];
 #pragma unroll
-      for (int c = 2; c < pf::BN; c += 2) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+      for (int k = 0; k < 8; ++k) {
+        float m = fmax3(__uint_as_float(sr[16 * k]), __uint_as_float(sr[16 * k + 1]),
+                        __uint_as_float(sr[16 * k + 2]));
+#pragma unroll
+        for (int e = 3; e < 15; e += 2)
+          m = fmax3(m, __uint_as_float(sr[16 * k + e]), __uint_as_float(sr[16 * k + e + 1]));
+        mxk[k] = fmaxf(m, __uint_as_float(sr[16 * k + 15]));
       }
-      const float mx = fmaxf(mx0, mx1);
+      const float mx = fmax3(fmax3(mxk[0], mxk[1], mxk[2]), fmax3(mxk[3], mxk[4], mxk[5]), fmaxf(mxk[6], mxk[7]));
       const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sl2;
       const bool grow = m_tile > m_run + pf::RESCALE_THRESHOLD;  // always true on the first tile
       if (__any_sync(0xffffffffu, grow)) {
@@ -399,27 +419,34 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           m_run = m_tile;
         }
       }
-      // P = 2^(s * scale_log2 - m) as bf16 pairs, written over the score columns
+      // P = 2^(s * scale_log2 - m) as bf16 pairs, written over the score
+      // columns in two halves so the first store overlaps the second half
       const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_run, -m_run);
-      float2 rs = make_float2(0.f, 0.f);
+      float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
       uint32_t* pw = sr;  // packed P overwrites the scores already consumed (c/2 < c)
 #pragma unroll
-      for (int c = 0; c < pf::BN; c += 2) {
-        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
-        float2 pr = ((c / 2) % pf::POLY_PAIR_EVERY == pf::POLY_PAIR_EVERY - 1)
-                        ? exp2_poly2(x)
-                        : make_float2(ex2(x.x), ex2(x.y));
-        if (diag) {  // masked keys: exactly 0 (the polynomial, or a zero scale, would not give it)
-          if (kv0 + c > limit) pr.x = 0.f;
-          if (kv0 + c + 1 > limit) pr.y = 0.f;
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int c = half * 64; c < half * 64 + 64; c += 2) {
+          const float2 x =
+              __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
+          float2 pr = (pf::POLY_PAIR_EVERY > 0 && (c / 2) % pf::POLY_PAIR_EVERY == pf::POLY_PAIR_EVERY - 1)
+                          ? exp2_poly2(x)
+                          : make_float2(ex2(x.x), ex2(x.y));
+          if (diag) {  // masked keys: exactly 0 (the polynomial, or a zero scale, would not give it)
+            if (kv0 + c > limit) pr.x = 0.f;
+            if (kv0 + c + 1 > limit) pr.y = 0.f;
+          }
+          rs[(c / 2) & 3] = __fadd2_rn(rs[(c / 2) & 3], pr);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(pr.x, pr.y);
+          pw[c / 2] = *reinterpret_cast<uint32_t*>(&h2);
         }
-        rs = __fadd2_rn(rs, pr);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(pr.x, pr.y);
-        pw[c / 2] = *reinterpret_cast<uint32_t*>(&h2);
+        tc::st_32x32b_x32(s_addr + half * 32, pw + half * 32);
       }
-      l_run += rs.x + rs.y;
-      tc::st_32x32b_x32(s_addr, pw);
-      tc::st_32x32b_x32(s_addr + 32, pw + 32);
+      const float2 r01 = __fadd2_rn(rs[0], rs[1]), r23 = __fadd2_rn(rs[2], rs[3]);
+      const float2 r = __fadd2_rn(r01, r23);
+      l_run += r.x + r.y;
       tc::wait_st();
       tc::fence_before_sync();
       __syncwarp();
