@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
-    ap.add_argument("--profile", default=None, choices=["decode", "split", "prefill", "write"],
+    ap.add_argument("--profile", default=None, choices=["decode", "decode_full", "split", "prefill", "write"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
@@ -167,6 +167,26 @@ def prefill_flops(case) -> int:
         vis = sum(L - Q + i + 1 for i in range(Q))
         f += 4 * case.D * vis * case.Hq
     return f
+
+
+# --------------------------------------------------------------------------- #
+# multi-rank aggregation                                                       #
+# --------------------------------------------------------------------------- #
+def max_over_ranks(values, dist=None):
+    """Element-wise maximum over all ranks: every device-timed figure is the
+    slowest rank's.  Ranks call this in the same order (a collective)."""
+    if dist is None:
+        return list(values)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(bytes_per_rank_step: int, world: int, ms_per_step: float) -> float:
+    """GB/s of the whole job: every rank runs its own replica of the step, so
+    the job moves world x the bytes in the slowest rank's step time."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
 
 
 # --------------------------------------------------------------------------- #
@@ -298,7 +318,16 @@ def profile_case(kind: str, launches: int = 3):
     import paged_kv_cache_477_b200 as pkv
     from paged_kv_cache_477_b200 import workloads as wl
     torch.cuda.set_device(0)
-    if kind in ("decode", "split", "write"):
+    if kind == "decode_full":
+        # the bench's own decode launch (Llama-3-8B-shaped, B=128): 2 GiB of K/V
+        c = wl.workload(WORKLOAD, device="cuda")
+        out = torch.empty_like(c.q)
+        ws = torch.empty(max(1, pkv.workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, 4096)), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(launches):
+            pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
+                                max_context_len=4096, workspace=ws)
+    elif kind in ("decode", "split", "write"):
         # 32 of the Llama-3-8B-shaped sequences: 512 MiB of K/V
         c = wl.make_case(B=32, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 32, seed=1003, device="cuda",
                          write_tokens=1)
@@ -427,15 +456,12 @@ def main():
 
     step_bytes = decode_bytes(case) + write_bytes(case)
     attn_bytes = decode_bytes(case)
-    if dist is not None:
-        tt = torch.tensor([elapsed_ms, e2e_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms, e2e_ms = tt.tolist()
+    elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dist)
 
     if rank == 0:
         ms_step = elapsed_ms / args.steps
-        value = world * step_bytes / (ms_step * 1e-3) / 1e9
-        e2e_val = world * step_bytes / (e2e_ms / args.steps * 1e-3) / 1e9
+        value = whole_job_rate(step_bytes, world, ms_step)
+        e2e_val = whole_job_rate(step_bytes, world, e2e_ms / args.steps)
         achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
         src = source_hash("decode_attn.cuh", "pkv_common.cuh")
         line = {
