@@ -254,20 +254,27 @@ def l2_flush_buffer():
     return torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
 
+def queue_ahead(ms: float = 5.0):
+    """Keep the device busy for about `ms` so the host can queue the calls
+    that follow; events around them then see device time only, not the
+    host's launch overhead."""
+    torch.cuda._sleep(int(ms * 2.0e6))  # ~2 GHz SM clock: cycles per ms
+
+
 def time_calls(fn, iters, flush=None):
-    """Per-call device times (ms) with CUDA events on the current stream."""
+    """Per-call device times (ms): CUDA events on the current stream around
+    each call, with every call queued before the first one runs."""
     st = torch.cuda.current_stream()
-    ts = []
-    for _ in range(iters):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    queue_ahead()
+    for e0, e1 in ev:
         if flush is not None:
             flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(st)
         fn()
         e1.record(st)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    return ts
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
 
 
 def extras(peaks):
@@ -404,6 +411,7 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
+        queue_ahead()
         t0.record(st)
         for i in range(args.steps):
             pkv.kv_cache_write(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping)

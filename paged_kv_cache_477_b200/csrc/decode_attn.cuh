@@ -10,16 +10,15 @@
 // the tensor cores.
 //
 // B200 design:
-//   * One CTA = (sequence b, a group of HG query heads sharing one kv head,
-//     a range of pages).  The HG query rows live in registers, so every K/V
+//   * Work is cut into segments: (sequence b, a group of HG query heads that
+//     share one kv head).  The HG query rows live in registers, so every K/V
 //     byte is read from HBM once per group (grouped-query reuse).
 //   * Every warp feeds itself: lane 0 issues 1-D bulk copies (cp.async.bulk)
 //     of whole pages -- a (block, kv head) page is one contiguous 4 KB (D=128)
 //     or 2 KB (D=64) run -- into the warp's own SW-stage shared-memory ring,
 //     completion tracked by one mbarrier per stage.  A warp refills a stage
 //     as soon as it has read it, so no cross-warp hand-off is needed and no
-//     warp is spent on copies.  Block-table entries are fetched 32 at a time,
-//     one chunk ahead.
+//     warp is spent on copies.
 //   * Two CTAs per SM (shared-memory carveout at its maximum) keep
 //     2 x NW x SW pages -- about 192 KB -- in flight per SM, which is what
 //     Little's law asks for at full HBM bandwidth.
@@ -27,14 +26,17 @@
 //     vectors each), so a warp covers 32/LPR rows per instruction and a dot
 //     product needs only log2(LPR) shuffle steps.  Products and P.V updates
 //     use packed fp32 (FFMA2) on element pairs.  Each lane keeps its own
-//     running max, sum and fp32 accumulator; lanes and warps merge once at
-//     the end by log-sum-exp.
-//   * Split mode (num_splits > 1): each CTA writes its normalised partial and
-//     its log2-domain log-sum-exp; lse_merge_kernel combines them.
+//     running max, sum and fp32 accumulator; lanes and warps merge by
+//     log-sum-exp when a segment (or a CTA's share of it) is done.
 //   * Shared-memory reads are conflict-free: for D=128 the 8 lanes of a row
 //     read 128 contiguous bytes per phase; for D=64 odd row groups read their
 //     two vectors in swapped order, and their q / accumulator registers are
 //     kept in that swapped order too.
+//   * One CTA per (segment, split of pages_per_split pages).  With one split
+//     the CTA writes the bf16 output itself; with several, each split writes
+//     a normalised fp32 partial and its log2-sum-exp, and lse_merge_kernel
+//     combines them.  The block scheduler hands CTAs to SMs as others finish,
+//     which absorbs ragged lengths and SMs that stream at different rates.
 #pragma once
 #include "pkv_common.cuh"
 
@@ -44,8 +46,8 @@ constexpr int kPageRows = 16;  // block_size supported by the attention kernels
 
 struct DecodeParams {
   __nv_bfloat16* out;            // [B][Hq][D]
-  float* o_part;                 // [B][Hq][C][D]   split mode
-  float* lse_part;               // [B][Hq][C]      split mode, log2 domain
+  float* o_part;                 // split partials [B][Hq][C][D]
+  float* lse_part;               // their log2-sum-exp [B][Hq][C]
   const __nv_bfloat16* q;        // [B][Hq][D]
   const unsigned char* k_cache;  // [NB][Hkv][16][D] bf16
   const unsigned char* v_cache;
@@ -60,20 +62,24 @@ struct DecodeParams {
   float scale_log2;              // scale * log2(e)
 };
 
-template <int D, int HG, int NW, int SW>
+// A ring stage holds PPS consecutive pages of one sequence: their K pages
+// side by side (ROWS = 16 * PPS contiguous key rows), then their V pages.
+template <int D, int HG, int NW, int SW, int PPS>
 struct DecodeShape {
   static_assert(D == 64 || D == 128, "head_dim");
   static constexpr int LPR = D / 16;              // lanes sharing one key row
   static constexpr int RPW = 32 / LPR;            // rows per warp step
-  static constexpr int TPL = kPageRows / RPW;     // rows per lane per page
+  static constexpr int ROWS = kPageRows * PPS;    // key rows per stage
+  static constexpr int TPL = ROWS / RPW;          // rows per lane per stage
   static constexpr int PAGE_BYTES = kPageRows * D * 2;
-  static constexpr int STAGE_BYTES = 2 * PAGE_BYTES;  // K page + V page
+  static constexpr int STAGE_BYTES = 2 * PPS * PAGE_BYTES;  // PPS K pages + PPS V pages
   static constexpr int THREADS = NW * 32;
   static constexpr int WARP_RING = SW * STAGE_BYTES;
   static constexpr int RING_BYTES = NW * WARP_RING;
-  // after its last page a warp reuses its own ring for the merge data
-  static constexpr int MERGE_BYTES = (HG * D + 2 * HG) * 4;
-  static_assert(MERGE_BYTES <= WARP_RING, "merge data must fit the warp's ring");
+  // one warp's merge data: acc [HG][D], m [HG], l [HG]; stride kept 16-byte aligned
+  static constexpr int MERGE_STRIDE = (HG * D + 2 * HG + 3) / 4 * 4;
+  static_assert(MERGE_STRIDE * 4 <= WARP_RING, "merge data must fit the warp's ring");
+  // rings, then barriers (merge data reuses each warp's ring)
   static constexpr int BAR_OFFSET = RING_BYTES;
   static constexpr int SMEM_BYTES = BAR_OFFSET + NW * SW * 8;
 };
@@ -82,10 +88,214 @@ __device__ __forceinline__ float2 widen2(uint32_t w) {
   return make_float2(bf16lo_to_f32(w), bf16hi_to_f32(w));
 }
 
-template <int D, int HG, int NW, int SW>
+// Per-lane running softmax state for HG query heads over the lane's 16
+// elements of D: running max m, running sum l, fp32 accumulator (8 pairs).
+template <int HG>
+struct LaneState {
+  float m[HG], l[HG];
+  float2 acc[HG][8];
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[h][e] = make_float2(0.f, 0.f);
+    }
+  }
+};
+
+// The lane's 16 q elements of each of the HG heads, as 8 pairs, pre-scaled.
+template <int D, int HG>
+__device__ __forceinline__ void load_q(float2 (&q2)[HG][8], const __nv_bfloat16* q_row0, int ch0,
+                                       int ch1, float scale_log2) {
+#pragma unroll
+  for (int h = 0; h < HG; ++h) {
+    const uint4* qrow = reinterpret_cast<const uint4*>(q_row0 + (size_t)h * D);
+    const uint4 a = __ldg(qrow + ch0), c = __ldg(qrow + ch1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) q2[h][e] = __fmul2_rn(widen2(w[e]), sc2);
+  }
+}
+
+// ROWS key rows (K at kp, V at vp, row stride D) into the lane state.  Rows
+// r >= nvalid (past the end of the sequence or of the copied pages) take no
+// part in the max and are never read from V.
+template <int D, int HG, int ROWS>
+__device__ __forceinline__ void attend_rows(LaneState<HG>& st, const float2 (&q2)[HG][8],
+                                            const unsigned char* kp, const unsigned char* vp,
+                                            int nvalid, int rg, int ch0, int ch1) {
+  constexpr int LPR = D / 16, RPW = 32 / LPR, TPL = ROWS / RPW;
+  float sc[TPL][HG];
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) {
+    const int r = rg + t * RPW;
+    const uint4* krow = reinterpret_cast<const uint4*>(kp + r * D * 2);
+    const uint4 ka = krow[ch0], kb = krow[ch1];
+    const float2 k2[8] = {widen2(ka.x), widen2(ka.y), widen2(ka.z), widen2(ka.w),
+                          widen2(kb.x), widen2(kb.y), widen2(kb.z), widen2(kb.w)};
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      float2 d = __fmul2_rn(q2[h][0], k2[0]);
+#pragma unroll
+      for (int e = 1; e < 8; ++e) d = __ffma2_rn(q2[h][e], k2[e], d);
+      sc[t][h] = d.x + d.y;
+    }
+  }
+#pragma unroll
+  for (int off = LPR / 2; off >= 1; off >>= 1)
+#pragma unroll
+    for (int t = 0; t < TPL; ++t)
+#pragma unroll
+      for (int h = 0; h < HG; ++h) sc[t][h] += __shfl_xor_sync(0xffffffffu, sc[t][h], off);
+
+  bool valid[TPL];
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) valid[t] = rg + t * RPW < nvalid;
+
+  float mp[HG];
+  bool grow = false;
+#pragma unroll
+  for (int h = 0; h < HG; ++h) {
+    mp[h] = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < TPL; ++t)
+      if (valid[t]) mp[h] = fmaxf(mp[h], sc[t][h]);
+    grow |= mp[h] > st.m[h];
+  }
+  if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      const float mn = fmaxf(st.m[h], mp[h]);
+      const float alpha = (mn == -INFINITY) ? 1.f : ex2(st.m[h] - mn);
+      st.m[h] = mn;
+      st.l[h] *= alpha;
+      const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) st.acc[h][e] = __fmul2_rn(st.acc[h][e], a2);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) {
+    if (!valid[t]) continue;  // canary / stale rows are never touched
+    const int r = rg + t * RPW;
+    const uint4* vrow = reinterpret_cast<const uint4*>(vp + r * D * 2);
+    const uint4 va = vrow[ch0], vb = vrow[ch1];
+    const float2 v2[8] = {widen2(va.x), widen2(va.y), widen2(va.z), widen2(va.w),
+                          widen2(vb.x), widen2(vb.y), widen2(vb.z), widen2(vb.w)};
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      const float pr = ex2(sc[t][h] - st.m[h]);
+      st.l[h] += pr;
+      const float2 pp = make_float2(pr, pr);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) st.acc[h][e] = __ffma2_rn(pp, v2[e], st.acc[h][e]);
+    }
+  }
+}
+
+// Merge the row groups of a warp (lanes holding the same D-slice) by
+// log-sum-exp; afterwards lanes 0..LPR-1 hold the warp's result in natural
+// element order.
+template <int D, int HG>
+__device__ __forceinline__ void warp_merge(LaneState<HG>& st) {
+  constexpr int LPR = D / 16;
+#pragma unroll
+  for (int off = LPR; off < 32; off <<= 1) {
+    const int flip = (D == 64 && off == LPR) ? 4 : 0;  // partner keeps the other order
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      const float mo = __shfl_xor_sync(0xffffffffu, st.m[h], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, st.l[h], off);
+      const float mn = fmaxf(st.m[h], mo);
+      const float a = (mn == -INFINITY) ? 0.f : ex2(st.m[h] - mn);
+      const float c = (mn == -INFINITY) ? 0.f : ex2(mo - mn);
+      float2 recv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        recv[e].x = __shfl_xor_sync(0xffffffffu, st.acc[h][e ^ flip].x, off);
+        recv[e].y = __shfl_xor_sync(0xffffffffu, st.acc[h][e ^ flip].y, off);
+      }
+      const float2 a2 = make_float2(a, a), c2 = make_float2(c, c);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) st.acc[h][e] = __ffma2_rn(st.acc[h][e], a2, __fmul2_rn(recv[e], c2));
+      st.l[h] = st.l[h] * a + lo * c;
+      st.m[h] = mn;
+    }
+  }
+}
+
+// Lanes 0..LPR-1 of a warp write its merged state to `mine` ([HG][D] acc,
+// [HG] m, [HG] l; 16-byte aligned).
+template <int D, int HG>
+__device__ __forceinline__ void warp_store(float* mine, const LaneState<HG>& st, int rg, int sub, int ch0,
+                                           int ch1) {
+  if (rg != 0) return;
+#pragma unroll
+  for (int h = 0; h < HG; ++h) {
+    float4* dst = reinterpret_cast<float4*>(mine + h * D);
+    dst[2 * ch0] = make_float4(st.acc[h][0].x, st.acc[h][0].y, st.acc[h][1].x, st.acc[h][1].y);
+    dst[2 * ch0 + 1] = make_float4(st.acc[h][2].x, st.acc[h][2].y, st.acc[h][3].x, st.acc[h][3].y);
+    dst[2 * ch1] = make_float4(st.acc[h][4].x, st.acc[h][4].y, st.acc[h][5].x, st.acc[h][5].y);
+    dst[2 * ch1 + 1] = make_float4(st.acc[h][6].x, st.acc[h][6].y, st.acc[h][7].x, st.acc[h][7].y);
+    if (sub == 0) {
+      mine[HG * D + h] = st.m[h];
+      mine[HG * D + HG + h] = st.l[h];
+    }
+  }
+}
+
+// Combine the NW warps' stored states (warp w at parts + w * stride floats)
+// and write either bf16 rows out_rows[h * D + d], or an fp32 partial
+// o_part[h * o_hstride + d] with its log2-sum-exp lse_part[h * lse_hstride].
+// The caller synchronises the CTA before and after.
+template <int D, int HG, int NW>
+__device__ __forceinline__ void cta_combine(const float* parts, int stride, __nv_bfloat16* out_rows,
+                                            float* o_part, size_t o_hstride, float* lse_part,
+                                            size_t lse_hstride) {
+  for (int idx = threadIdx.x; idx < HG * D; idx += NW * 32) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, parts[w * stride + HG * D + h]);
+    float Ls = 0.f, A = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float* part = parts + w * stride;
+      const float mw = part[HG * D + h];
+      if (mw == -INFINITY) continue;  // this warp saw no valid row
+      const float wt = ex2(mw - M);
+      Ls = fmaf(part[HG * D + HG + h], wt, Ls);
+      A = fmaf(part[h * D + d], wt, A);
+    }
+    if (out_rows != nullptr) {
+      out_rows[idx] = __float2bfloat16_rn(Ls > 0.f ? A / Ls : 0.f);
+    } else {
+      o_part[h * o_hstride + d] = Ls > 0.f ? A / Ls : 0.f;
+      if (d == 0) lse_part[h * lse_hstride] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
+    }
+  }
+}
+
+// Wait for the last issued use of every stage of a warp ring (only needed
+// when a wait ran out and pages were left unconsumed).
+template <int SW>
+__device__ __forceinline__ void drain_ring(uint32_t wbar, int issued) {
+  for (int s = 0; s < SW && s < issued; ++s) {
+    const int last = s + ((issued - 1 - s) / SW) * SW;
+    mbar_wait(wbar + 8 * s, (last / SW) & 1);
+  }
+}
+
+// ============================================================================
+// One CTA per (split, head group, sequence).
+// ============================================================================
+template <int D, int HG, int NW, int SW, int PPS>
 __global__ void __launch_bounds__(NW * 32)
     decode_attn_kernel(const __grid_constant__ DecodeParams p) {
-  using S = DecodeShape<D, HG, NW, SW>;
+  using S = DecodeShape<D, HG, NW, SW, PPS>;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int split = blockIdx.x, hsub = blockIdx.y, b = blockIdx.z;
@@ -93,13 +303,35 @@ __global__ void __launch_bounds__(NW * 32)
   const int head0 = kvh * p.G + (hsub % p.nsub) * HG;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  const int pg0 = split * p.pages_per_split;
+  // The CTA's pages are cut into units of PPS consecutive pages, one unit per
+  // ring stage; unit j of this warp is unit u = warp + j * NW, pages
+  // pg0 + u * PPS + i.  Lane l of a chunk holds the block-table entries of
+  // unit j = 32 * chunk + l.  The first two chunks are loaded together with
+  // the context length (bounded by the table row and the split, not by the
+  // length), so the CTA waits for one load latency before its first copy
+  // instead of two.  Entries are validated where they are used.
+  const int32_t* btrow = p.block_tables + (size_t)b * p.MB;
+  struct Entries {
+    int blk[PPS];
+  };
+  auto load_raw = [&](int c) {
+    Entries e;
+#pragma unroll
+    for (int i = 0; i < PPS; ++i) {
+      const int w = (warp + (c * 32 + lane) * NW) * PPS + i;  // page index within the split
+      e.blk[i] = (w < p.pages_per_split && pg0 + w < p.MB) ? __ldg(btrow + pg0 + w) : 0;
+    }
+    return e;
+  };
   int L = __ldg(p.context_lens + b);
+  const Entries raw0 = load_raw(0);
+  Entries bt_nxt = load_raw(1);
   if (L < 0 || L > p.cap_tokens) {
     if (threadIdx.x == 0) set_error(PKV_ERR_BOUNDS);
     L = L < 0 ? 0 : p.cap_tokens;
   }
   const int npages = (L + kPageRows - 1) / kPageRows;
-  const int pg0 = split * p.pages_per_split;
   const int n = min(npages - pg0, p.pages_per_split);  // pages of this CTA
   // A wait that ran out earlier leaves a sticky error: do no more work until
   // the host has read and cleared it.  One thread reads the word so the whole
@@ -117,8 +349,9 @@ __global__ void __launch_bounds__(NW * 32)
     return;
   }
 
-  // ------------------------------------------------ this warp's page stream --
-  const int my_n = warp < n ? (n - warp + NW - 1) / NW : 0;  // pages warp, warp+NW, ...
+  // ------------------------------------------------ this warp's unit stream --
+  const int nu = (n + PPS - 1) / PPS;                           // units of this CTA
+  const int my_n = warp < nu ? (nu - warp + NW - 1) / NW : 0;  // units warp, warp+NW, ...
   const uint32_t wring = smem_addr(smem) + warp * S::WARP_RING;
   const uint32_t wbar = smem_addr(smem) + S::BAR_OFFSET + warp * SW * 8;
   unsigned char* wring_ptr = smem + warp * S::WARP_RING;
@@ -128,37 +361,42 @@ __global__ void __launch_bounds__(NW * 32)
   }
   __syncwarp();
 
-  const int32_t* btw = p.block_tables + (size_t)b * p.MB + pg0 + warp;  // entry of page j: btw[j*NW]
-  auto load_chunk = [&](int c) {
+  auto validate = [&](Entries e, int c) {  // entries of pages this warp reads must lie in the pool
     const int j = c * 32 + lane;
-    int blk = 0;
-    if (j < my_n) {
-      blk = __ldg(btw + (size_t)j * NW);
-      if (blk < 0 || blk >= p.NB) {
+#pragma unroll
+    for (int i = 0; i < PPS; ++i)
+      if (j < my_n && (warp + j * NW) * PPS + i < n && (e.blk[i] < 0 || e.blk[i] >= p.NB)) {
         set_error(PKV_ERR_BOUNDS);
-        blk = 0;  // keep every copy inside the pool
+        e.blk[i] = 0;  // keep every copy inside the pool
       }
-    }
-    return blk;
+    return e;
   };
-  int bt_cur = load_chunk(0), bt_nxt = load_chunk(1), chunk = 0;
+  Entries bt_cur = validate(raw0, 0);
+  int chunk = 0;
   const uint64_t pol = policy_evict_first();  // every page is read once
   int issued = 0;
-  auto issue_next = [&]() {  // warp-uniform; pages are issued in order
+  auto issue_next = [&]() {  // warp-uniform; units are issued in order
     const int k = issued;
     if ((k >> 5) != chunk) {
-      bt_cur = bt_nxt;
       chunk = k >> 5;
-      bt_nxt = load_chunk(chunk + 1);
+      bt_cur = validate(bt_nxt, chunk);
+      bt_nxt = load_raw(chunk + 1);
     }
-    const int blk = __shfl_sync(0xffffffffu, bt_cur, k & 31);
+    const int np = min(PPS, n - (warp + k * NW) * PPS);  // pages of this unit (>= 1)
+    int blk[PPS];
+#pragma unroll
+    for (int i = 0; i < PPS; ++i) blk[i] = __shfl_sync(0xffffffffu, bt_cur.blk[i], k & 31);
     if (lane == 0) {
       const int s = k % SW;
-      const size_t off = ((size_t)blk * p.Hkv + kvh) * S::PAGE_BYTES;
-      mbar_arrive_expect_tx(wbar + 8 * s, S::STAGE_BYTES);
-      bulk_g2s_hint(wring + s * S::STAGE_BYTES, p.k_cache + off, S::PAGE_BYTES, wbar + 8 * s, pol);
-      bulk_g2s_hint(wring + s * S::STAGE_BYTES + S::PAGE_BYTES, p.v_cache + off, S::PAGE_BYTES,
-                    wbar + 8 * s, pol);
+      const uint32_t stage = wring + s * S::STAGE_BYTES;
+      mbar_arrive_expect_tx(wbar + 8 * s, np * 2 * S::PAGE_BYTES);
+#pragma unroll
+      for (int i = 0; i < PPS; ++i) {
+        if (i >= np) break;
+        const size_t off = ((size_t)blk[i] * p.Hkv + kvh) * S::PAGE_BYTES;
+        bulk_g2s_hint(stage + i * S::PAGE_BYTES, p.k_cache + off, S::PAGE_BYTES, wbar + 8 * s, pol);
+        bulk_g2s_hint(stage + (PPS + i) * S::PAGE_BYTES, p.v_cache + off, S::PAGE_BYTES, wbar + 8 * s, pol);
+      }
     }
     ++issued;
   };
@@ -169,29 +407,14 @@ __global__ void __launch_bounds__(NW * 32)
   const int swap = (D == 64) ? (rg & 1) : 0;
   const int ch0 = sub + S::LPR * swap;        // 16-byte vector held in slot 0
   const int ch1 = sub + S::LPR * (swap ^ 1);  // and in slot 1
+  float2 q2[HG][8];
+  load_q<D, HG>(q2, p.q + ((size_t)b * p.Hq + head0) * D, ch0, ch1, p.scale_log2);
+  LaneState<HG> st;
+  st.reset();
 
-  float2 q2[HG][8];  // the lane's 16 q elements as 8 pairs, pre-scaled
-#pragma unroll
-  for (int h = 0; h < HG; ++h) {
-    const uint4* qrow = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + head0 + h) * D);
-    const uint4 a = __ldg(qrow + ch0), c = __ldg(qrow + ch1);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) q2[h][e] = __fmul2_rn(widen2(w[e]), sc2);
-  }
-
-  float m[HG], l[HG];
-  float2 acc2[HG][8];
-#pragma unroll
-  for (int h = 0; h < HG; ++h) {
-    m[h] = -INFINITY;
-    l[h] = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc2[h][e] = make_float2(0.f, 0.f);
-  }
-
-  const int L_local = L - pg0 * kPageRows;  // valid rows counted from this CTA's first page
+  // valid rows counted from this CTA's first page: the sequence's, and no
+  // further than the CTA's own pages
+  const int rows_cta = min(L - pg0 * kPageRows, n * kPageRows);
   int done = 0;
   for (int j = 0; j < my_n; ++j, ++done) {
     const int s = j % SW;
@@ -200,75 +423,8 @@ __global__ void __launch_bounds__(NW * 32)
     const bool ok = mbar_wait(wbar + 8 * s, (j / SW) & 1);
     if (!__all_sync(0xffffffffu, ok)) break;
     const unsigned char* kp = wring_ptr + s * S::STAGE_BYTES;
-    const unsigned char* vp = kp + S::PAGE_BYTES;
-    const int row0 = (warp + j * NW) * kPageRows;
-
-    float sc[S::TPL][HG];
-#pragma unroll
-    for (int t = 0; t < S::TPL; ++t) {
-      const int r = rg + t * S::RPW;
-      const uint4* krow = reinterpret_cast<const uint4*>(kp + r * D * 2);
-      const uint4 ka = krow[ch0], kb = krow[ch1];
-      const float2 k2[8] = {widen2(ka.x), widen2(ka.y), widen2(ka.z), widen2(ka.w),
-                            widen2(kb.x), widen2(kb.y), widen2(kb.z), widen2(kb.w)};
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        float2 d = __fmul2_rn(q2[h][0], k2[0]);
-#pragma unroll
-        for (int e = 1; e < 8; ++e) d = __ffma2_rn(q2[h][e], k2[e], d);
-        sc[t][h] = d.x + d.y;
-      }
-    }
-#pragma unroll
-    for (int off = S::LPR / 2; off >= 1; off >>= 1)
-#pragma unroll
-      for (int t = 0; t < S::TPL; ++t)
-#pragma unroll
-        for (int h = 0; h < HG; ++h) sc[t][h] += __shfl_xor_sync(0xffffffffu, sc[t][h], off);
-
-    bool valid[S::TPL];
-#pragma unroll
-    for (int t = 0; t < S::TPL; ++t) valid[t] = row0 + rg + t * S::RPW < L_local;
-
-    float mp[HG];
-    bool grow = false;
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      mp[h] = -INFINITY;
-#pragma unroll
-      for (int t = 0; t < S::TPL; ++t)
-        if (valid[t]) mp[h] = fmaxf(mp[h], sc[t][h]);
-      grow |= mp[h] > m[h];
-    }
-    if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float mn = fmaxf(m[h], mp[h]);
-        const float alpha = (mn == -INFINITY) ? 1.f : ex2(m[h] - mn);
-        m[h] = mn;
-        l[h] *= alpha;
-        const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc2[h][e] = __fmul2_rn(acc2[h][e], a2);
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < S::TPL; ++t) {
-      if (!valid[t]) continue;  // canary / stale rows are never touched
-      const int r = rg + t * S::RPW;
-      const uint4* vrow = reinterpret_cast<const uint4*>(vp + r * D * 2);
-      const uint4 va = vrow[ch0], vb = vrow[ch1];
-      const float2 v2[8] = {widen2(va.x), widen2(va.y), widen2(va.z), widen2(va.w),
-                            widen2(vb.x), widen2(vb.y), widen2(vb.z), widen2(vb.w)};
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        const float pr = ex2(sc[t][h] - m[h]);
-        l[h] += pr;
-        const float2 pp = make_float2(pr, pr);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc2[h][e] = __ffma2_rn(pp, v2[e], acc2[h][e]);
-      }
-    }
+    attend_rows<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES, rows_cta - (warp + j * NW) * S::ROWS, rg,
+                                ch0, ch1);
     if (issued < my_n) {
       // the stage just read is refilled: order the generic-proxy reads of all
       // lanes before the copy engine's writes
@@ -278,85 +434,22 @@ __global__ void __launch_bounds__(NW * 32)
     }
   }
   // Never reuse or leave the ring while one of this warp's copies may still
-  // land in it (only possible after a timeout): wait for the last issued use
-  // of every stage.
-  if (done < issued && lane == 0) {
-    for (int s = 0; s < SW && s < issued; ++s) {
-      const int last = s + ((issued - 1 - s) / SW) * SW;
-      mbar_wait(wbar + 8 * s, (last / SW) & 1);
-    }
-  }
+  // land in it (only possible after a timeout).
+  if (done < issued && lane == 0) drain_ring<SW>(wbar, issued);
   __syncwarp();
 
-  // ---- merge the row groups of this warp (lanes with the same D-slice) ----
-#pragma unroll
-  for (int off = S::LPR; off < 32; off <<= 1) {
-    const int flip = (D == 64 && off == S::LPR) ? 4 : 0;  // partner keeps the other order
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[h], off);
-      const float lo = __shfl_xor_sync(0xffffffffu, l[h], off);
-      const float mn = fmaxf(m[h], mo);
-      const float a = (mn == -INFINITY) ? 0.f : ex2(m[h] - mn);
-      const float c = (mn == -INFINITY) ? 0.f : ex2(mo - mn);
-      float2 recv[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        recv[e].x = __shfl_xor_sync(0xffffffffu, acc2[h][e ^ flip].x, off);
-        recv[e].y = __shfl_xor_sync(0xffffffffu, acc2[h][e ^ flip].y, off);
-      }
-      const float2 a2 = make_float2(a, a), c2 = make_float2(c, c);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc2[h][e] = __ffma2_rn(acc2[h][e], a2, __fmul2_rn(recv[e], c2));
-      l[h] = l[h] * a + lo * c;
-      m[h] = mn;
-    }
-  }
-
-  // ---- merge the warps through shared memory (each warp's own ring) -------
-  {
-    float* mine = reinterpret_cast<float*>(wring_ptr);  // [HG][D] acc, [HG] m, [HG] l
-    if (rg == 0) {  // lanes 0..LPR-1 hold the warp's result in natural order
-#pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        float4* dst = reinterpret_cast<float4*>(mine + h * D);
-        dst[2 * ch0] = make_float4(acc2[h][0].x, acc2[h][0].y, acc2[h][1].x, acc2[h][1].y);
-        dst[2 * ch0 + 1] = make_float4(acc2[h][2].x, acc2[h][2].y, acc2[h][3].x, acc2[h][3].y);
-        dst[2 * ch1] = make_float4(acc2[h][4].x, acc2[h][4].y, acc2[h][5].x, acc2[h][5].y);
-        dst[2 * ch1 + 1] = make_float4(acc2[h][6].x, acc2[h][6].y, acc2[h][7].x, acc2[h][7].y);
-        if (sub == 0) {
-          mine[HG * D + h] = m[h];
-          mine[HG * D + HG + h] = l[h];
-        }
-      }
-    }
-  }
+  warp_merge<D, HG>(st);
+  // after its last page a warp reuses its own ring for its merge data
+  warp_store<D, HG>(reinterpret_cast<float*>(wring_ptr), st, rg, sub, ch0, ch1);
   __syncthreads();
-  for (int idx = threadIdx.x; idx < HG * D; idx += NW * 32) {
-    const int h = idx / D, d = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w)
-      M = fmaxf(M, reinterpret_cast<const float*>(smem + w * S::WARP_RING)[HG * D + h]);
-    float Ls = 0.f, A = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float* part = reinterpret_cast<const float*>(smem + w * S::WARP_RING);
-      const float mw = part[HG * D + h];
-      if (mw == -INFINITY) continue;  // this warp saw no valid row
-      const float wt = ex2(mw - M);
-      Ls = fmaf(part[HG * D + HG + h], wt, Ls);
-      A = fmaf(part[h * D + d], wt, A);
-    }
-    const size_t row = (size_t)b * p.Hq + head0 + h;
-    if (p.num_splits == 1) {
-      p.out[row * D + d] = __float2bfloat16_rn(Ls > 0.f ? A / Ls : 0.f);
-    } else {
-      const size_t prow = row * p.num_splits + split;
-      p.o_part[prow * D + d] = Ls > 0.f ? A / Ls : 0.f;
-      if (d == 0) p.lse_part[prow] = Ls > 0.f ? M + log2f(Ls) : -INFINITY;
-    }
-  }
+  const size_t row = (size_t)b * p.Hq + head0;
+  const float* parts = reinterpret_cast<const float*>(smem);
+  if (p.num_splits == 1)
+    cta_combine<D, HG, NW>(parts, S::WARP_RING / 4, p.out + row * D, nullptr, 0, nullptr, 0);
+  else  // head h of this split: o_part[((row + h) * C + split) * D + d], lse_part[(row + h) * C + split]
+    cta_combine<D, HG, NW>(parts, S::WARP_RING / 4, nullptr, p.o_part + (row * p.num_splits + split) * D,
+                           (size_t)p.num_splits * D, p.lse_part + row * p.num_splits + split,
+                           (size_t)p.num_splits);
 }
 
 // ----------------------------------------------------------------------------

@@ -50,16 +50,18 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ----------------------------------------------------------------- decode --
 constexpr int kDecodeWarps = 4;
-// stages per warp: 3 x 8 KB (D=128) or 6 x 4 KB (D=64) -> 96 KB of pages in
-// flight per CTA, two CTAs per SM
-constexpr int stages_for(int D) { return D == 128 ? 3 : 6; }
+// pages per ring stage: two for D=64, so a stage is 32 key rows and a lane
+// works on four rows per step whatever D is
+constexpr int pages_per_stage(int D) { return D == 128 ? 1 : 2; }
+// stages per warp: 3 x 8 KB -> 96 KB of pages in flight per CTA, two CTAs per SM
+constexpr int stages_for(int D) { return 3; }
 
 template <int D, int HG>
-using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D)>;
+using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D), pages_per_stage(D)>;
 
 template <int D, int HG>
 struct DecodeKernel {
-  static constexpr auto fn = pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D)>;
+  static constexpr auto fn = pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D), pages_per_stage(D)>;
   // set the dynamic shared-memory limit once per device; return CTAs per SM
   static int prepare(int dev) {
     static int occ[kMaxDevices] = {0};
@@ -117,11 +119,17 @@ size_t split_ws_bytes(int32_t B, int32_t Hq, int32_t D, int32_t C) {
   return round256(rows * D * sizeof(float)) + round256(rows * sizeof(float));
 }
 
-// Host-only choice of the split count.  Aim for at least four waves of CTAs
-// so the block scheduler can balance ragged lengths, but keep every split at
-// least kMinSplitPages pages long so per-CTA set-up stays amortised.
-constexpr int kMinSplitPages = 32;
-constexpr int kTargetWaves = 4;
+// Host-only choice of the split size.  Every CTA pays a few microseconds to
+// start its copy stream and to merge at the end, so splits are kept long; a
+// CTA streams ~40 GB/s when its SM is shared, so 96 pages (0.4-0.8 MB) take
+// 10-20 us.  When the head groups alone give about three waves of CTAs the
+// block scheduler balances them without splitting, unless a context can be
+// long enough to leave one CTA running alone at the end: splits of up to
+// kSplitPagesMany pages then.  The host sees only max_context_len, not the
+// lengths themselves, so the rule is written for the longest context.
+constexpr int kSplitPages = 96;
+constexpr int kSplitPagesMany = 256;
+constexpr int kWavesNoSplit = 3;
 
 DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, int32_t bs,
                      int32_t hint) {
@@ -132,11 +140,11 @@ DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, 
   const int dev = current_device();
   const int occ = std::max(1, decode_occupancy(D, HG, dev));
   const int64_t slots = (int64_t)device_sm_count(dev) * occ;
-  if (units <= 0 || max_pages <= kMinSplitPages) return pl;
-  int64_t C = (kTargetWaves * slots + units - 1) / units;
-  C = std::min<int64_t>(C, max_pages / kMinSplitPages);
+  if (units <= 0) return pl;
+  const int target = units >= kWavesNoSplit * slots ? kSplitPagesMany : kSplitPages;
+  const int C = (max_pages + target - 1) / target;
   if (C <= 1) return pl;
-  const int pps = (int)((max_pages + C - 1) / C);
+  const int pps = (max_pages + C - 1) / C;  // equal splits no longer than the target
   pl.pages_per_split = pps;
   pl.num_splits = (max_pages + pps - 1) / pps;
   pl.workspace = split_ws_bytes(B, Hq, D, pl.num_splits);

@@ -88,6 +88,9 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O when the max
 #endif
 // one column pair in POLY_PAIR_EVERY takes the FMA-pipe exp2 (0: none)
 constexpr int POLY_PAIR_EVERY = PKV_PREFILL_POLY_EVERY;
+__host__ __device__ constexpr bool poly_pair(int pair) {
+  return POLY_PAIR_EVERY > 0 && pair % (POLY_PAIR_EVERY > 0 ? POLY_PAIR_EVERY : 1) == POLY_PAIR_EVERY - 1;
+}
 constexpr int REGS_LAUNCH = 168;    // 65536 / 384 rounded down to a multiple of 8
 constexpr int REGS_LOW = 64;        // load / MMA / allocator warpgroup
 constexpr int REGS_HIGH = 216;      // softmax warpgroups
@@ -124,7 +127,7 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  extern __shared__ __align__(16) unsigned char smem_raw[];  // base aligned to 1 KB by hand below
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sbase = smem_raw + (base - raw);
@@ -431,7 +434,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         for (int c = half * 64; c < half * 64 + 64; c += 2) {
           const float2 x =
               __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
-          float2 pr = (pf::POLY_PAIR_EVERY > 0 && (c / 2) % pf::POLY_PAIR_EVERY == pf::POLY_PAIR_EVERY - 1)
+          float2 pr = pf::poly_pair(c / 2)
                           ? exp2_poly2(x)
                           : make_float2(ex2(x.x), ex2(x.y));
           if (diag) {  // masked keys: exactly 0 (the polynomial, or a zero scale, would not give it)

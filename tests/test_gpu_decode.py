@@ -206,3 +206,32 @@ def test_bounded_wait_gives_up_and_context_survives():
                               case.scale)
     assert_close(out, HostCase(case).decode_ref(), "after timeout")
     _no_device_error()
+
+
+def test_decode_many_short_sequences():
+    """B = 2100 short sequences (one CTA per head group, several waves),
+    including empty and one-token contexts."""
+    g = torch.Generator().manual_seed(77)
+    lens = torch.randint(0, 40, (2100,), generator=g).tolist()
+    case = _decode_case(lens, 8, 2, 64, seed=77)
+    ref = HostCase(case).decode_ref()
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale)
+    assert_close(out, ref, "B=2100")
+    _no_device_error()
+
+
+def test_decode_ragged_batch_auto_and_split_agree():
+    """A ragged batch (empty, one-page and long contexts) through the automatic
+    plan and an explicit split size, every row checked."""
+    lens = [5000, 3, 0, 17, 1200, 4096, 640, 33] * 3
+    case = _decode_case(lens, 32, 8, 128, seed=78)
+    ref = HostCase(case).decode_ref()
+    auto = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                               case.scale)
+    assert_close(auto, ref, "auto")
+    split = pkv.paged_attention_split(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                      case.context_lens, case.scale, pages_per_split=64)
+    assert pkv.last_launch_count() == 2
+    assert_close(split, ref, "split pps=64")
+    _no_device_error()
