@@ -49,7 +49,8 @@ def parse():
     ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
-    ap.add_argument("--profile", default=None, choices=["decode", "decode_full", "split", "prefill", "write"],
+    ap.add_argument("--profile", default=None,
+                    choices=["decode", "decode_full", "decode_d64", "split", "prefill", "write"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
@@ -192,56 +193,81 @@ def whole_job_rate(bytes_per_rank_step: int, world: int, ms_per_step: float) -> 
 # --------------------------------------------------------------------------- #
 # the oracle on host cores                                                     #
 # --------------------------------------------------------------------------- #
-def oracle_decode_rate(seconds: float):
-    """Oracle decode over a bounded sample of llama3_8b_decode-shaped sequences.
-    Returns (GB/s, cores, sample description)."""
-    import oracle
-    from paged_kv_cache_477_b200 import workloads as wl
-    from paged_kv_cache_477_b200.workloads import bf16_bits
-    orc = oracle.get()
-    spec = wl.WORKLOADS[WORKLOAD]
+class OracleSample:
+    """A bounded sample of the bench workload for the fp64 oracle: the first n
+    of its sequences, n chosen so one oracle pass takes about `seconds`."""
 
-    def run(nseq):
-        c = wl.make_case(B=nseq, Hq=spec["Hq"], Hkv=spec["Hkv"], D=spec["D"], bs=spec["bs"],
-                         lens=[spec["lens"][0]] * nseq, seed=spec["seed"], device="cpu")
-        q, k, v = bf16_bits(c.q), bf16_bits(c.k_cache), bf16_bits(c.v_cache)
-        bt, cl = c.block_tables.numpy(), c.context_lens.numpy()
+    def __init__(self, seconds: float):
+        import oracle
+        from paged_kv_cache_477_b200 import workloads as wl
+        self.orc = oracle.get()
+        self.spec = wl.WORKLOADS[WORKLOAD]
+        self.args, _ = self._case(1)
+        t1 = self.run()
+        self.n = int(max(1, min(self.spec["B"], seconds / max(t1, 1e-3))))
+        self.args, self.nbytes = self._case(self.n)
+
+    def _case(self, nseq):
+        """Host arrays of the sample: (write args or None, attention args), bytes."""
+        from paged_kv_cache_477_b200 import workloads as wl
+        from paged_kv_cache_477_b200.workloads import bf16_bits
+        sp = self.spec
+        c = wl.make_case(B=nseq, Hq=sp["Hq"], Hkv=sp["Hkv"], D=sp["D"], bs=sp["bs"], lens=[sp["lens"][0]] * nseq,
+                         seed=sp["seed"], device="cpu", write_tokens=sp.get("write_tokens", 0))
+        k, v = bf16_bits(c.k_cache).copy(), bf16_bits(c.v_cache).copy()
+        write = None
+        if c.new_key is not None:
+            write = (bf16_bits(c.new_key), bf16_bits(c.new_value), k, v, c.slot_mapping.numpy())
+        attn = (bf16_bits(c.q), k, v, c.block_tables.numpy(), c.context_lens.numpy(), c.scale)
+        return (write, attn), decode_bytes(c) + (write_bytes(c) if write is not None else 0)
+
+    def run(self) -> float:
+        """One step of the bench on the host: the cache write, then decode."""
+        write, attn = self.args
         t0 = time.perf_counter()
-        orc.paged_attention(q, k, v, bt, cl, c.scale)
-        return time.perf_counter() - t0, decode_bytes(c)
+        if write is not None:
+            self.orc.kv_cache_write(*write)
+        self.orc.paged_attention(*attn)
+        return time.perf_counter() - t0
 
-    t1, _ = run(1)
-    n = int(max(1, min(spec["B"], seconds / max(t1, 1e-3))))
-    t, nbytes = run(n)
-    desc = (f"fp64 C oracle decode of {n} of the {spec['B']} sequences (ctx {spec['lens'][0]}, "
-            f"{spec['Hq']} q / {spec['Hkv']} kv heads, D={spec['D']}), OpenMP, {t:.1f} s")
-    return nbytes / t / 1e9, orc.num_threads(), desc, t
+    def describe(self, reps: int, secs: float) -> str:
+        sp = self.spec
+        return (f"fp64 C oracle decode of {self.n} of the {sp['B']} sequences (ctx {sp['lens'][0]}, "
+                f"{sp['Hq']} q / {sp['Hkv']} kv heads, D={sp['D']}) x {reps}, OpenMP, {secs:.1f} s")
+
+
+def oracle_decode_rate(seconds: float):
+    """Oracle decode rate on the host cores, repeated passes over a bounded
+    sample for about `seconds`.  Returns (GB/s, cores, sample description)."""
+    smp = OracleSample(min(seconds, 5.0))
+    t, reps = smp.run(), 1
+    while t < seconds:
+        t, reps = t + smp.run(), reps + 1
+    return smp.nbytes * reps / t / 1e9, smp.orc.num_threads(), smp.describe(reps, t)
 
 
 # --------------------------------------------------------------------------- #
 # reference arm: the oracle, as it stands, on host cores                       #
 # --------------------------------------------------------------------------- #
 def run_reference(args, rank, world):
+    """One step = one oracle pass over a bounded sample of the workload."""
     if rank != 0:
         return
     per_step = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    smp = OracleSample(per_step)
     for _ in range(args.warmup):
-        oracle_decode_rate(per_step)
-    vals, secs = [], 0.0
-    desc, cores = "", 1
-    for _ in range(args.steps):
-        v, cores, desc, t = oracle_decode_rate(per_step)
-        vals.append(v)
-        secs += t
-    value = statistics.median(vals)
+        smp.run()
+    ts = [smp.run() for _ in range(args.steps)]
+    secs = sum(ts)
+    value = smp.nbytes * args.steps / secs / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{WORKLOAD} (bounded sample per step)", "parallelism": "host cores"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": smp.orc.num_threads(),
+                         "kind": "oracle", "sample": smp.describe(args.steps, secs)},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -334,6 +360,13 @@ def profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
                                 max_context_len=4096, workspace=ws)
+    elif kind == "decode_d64":
+        # the Llama-3.2-1B-shaped decode (D=64): 300 MB of K/V
+        c = wl.workload("llama32_1b_decode", device="cuda")
+        out = torch.empty_like(c.q)
+        for _ in range(launches):
+            pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
+                                max_context_len=4096)
     elif kind in ("decode", "split", "write"):
         # 32 of the Llama-3-8B-shaped sequences: 512 MiB of K/V
         c = wl.make_case(B=32, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 32, seed=1003, device="cuda",
@@ -494,7 +527,7 @@ def main():
         if not args.no_extras and world == 1:
             line["extras"] = extras(peaks)
         if world == 1:
-            v, cores, desc, _ = oracle_decode_rate(args.cpu_seconds)
+            v, cores, desc = oracle_decode_rate(args.cpu_seconds)
             line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                     "sample": desc}
         print(json.dumps(line), flush=True)
