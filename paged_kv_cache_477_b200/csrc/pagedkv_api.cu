@@ -458,7 +458,12 @@ pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* 
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NB = NB; p.MB = MB; p.G = G; p.sumQ = sumQ;
   p.scale_log2 = scale * 1.4426950408889634f;
   const int ppc = pkv::pf::NQT * (pkv::pf::BM / G);  // query positions per CTA
-  dim3 grid((max_q_len + ppc - 1) / ppc, Hkv, B);
+  // Query tiles are the slowest grid dimension, launched last tile first: a
+  // later tile sees more keys, so the longest CTAs start in the first wave
+  // and the shortest fill the last one.
+  const int nct = (max_q_len + ppc - 1) / ppc;
+  if (nct > 65535 || B > 65535) return PKV_ERR_UNSUPPORTED;
+  dim3 grid(Hkv, B, nct);
   pkv::prefill_attn_kernel<<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
       p, tm_q, tm_k, tm_v);
   pkv_status s = launch_status();

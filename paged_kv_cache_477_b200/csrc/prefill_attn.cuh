@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sbase = smem_raw + (base - raw);
 
-  const int ct = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int kvh = blockIdx.x, b = blockIdx.y, ct = gridDim.z - 1 - blockIdx.z;  // last query tile first
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G, PPT = pf::BM / G;  // query positions per tile
 
@@ -260,11 +260,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           mbar_wait(bar(pf::B_VFULL + s), (last / pf::VSTAGES) & 1);
         }
       }
-    } else if (warp == 1) {
+    } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------- MMA ------
+      // One thread: it alone waits on the barriers it needs and issues every
+      // MMA and commit, so no warp-wide vote sits between two MMA groups.
       constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(pf::BM, pf::BN, false, false);
       constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(pf::BM, pf::D, false, true);
-      bool ok = __all_sync(0xffffffffu, mbar_wait(bar(pf::B_Q), 0));
+      bool ok = mbar_wait(bar(pf::B_Q), 0);
       // the page holding the sequence's last key, if it is only partly valid
       const int tail_rows = L % 16;
       const int tail_page = (L - 1) / 16;
@@ -277,54 +279,47 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       constexpr uint32_t TILE16 = pf::TILE_BYTES >> 4;
       auto qk = [&](int i, int j) {  // S_i = Q_i K_j^T
         const int ks = j % pf::KSTAGES;
-        if (lane == 0) {
-          const uint64_t dq = desc_q + i * TILE16, dk = desc_k + ks * TILE16;
-          const uint32_t d_s = tmem + i * pf::TILE_COLS;
+        const uint64_t dq = desc_q + i * TILE16, dk = desc_k + ks * TILE16;
+        const uint32_t d_s = tmem + i * pf::TILE_COLS;
 #pragma unroll
-          for (int kk = 0; kk < pf::D / 16; ++kk) {
-            const uint32_t off16 = ((kk >> 2) * pf::HALF_BYTES + (kk & 3) * 32) >> 4;
-            tc::mma_ss(d_s, dq + off16, dk + off16, IDESC_S, kk > 0 ? 1u : 0u);
-          }
-          tc::commit(bar(pf::B_SFULL + i));
-          if (i == pf::NQT - 1) tc::commit(bar(pf::B_KEMPTY + ks));
+        for (int kk = 0; kk < pf::D / 16; ++kk) {
+          const uint32_t off16 = ((kk >> 2) * pf::HALF_BYTES + (kk & 3) * 32) >> 4;
+          tc::mma_ss(d_s, dq + off16, dk + off16, IDESC_S, kk > 0 ? 1u : 0u);
         }
-        __syncwarp();
+        tc::commit(bar(pf::B_SFULL + i));
+        if (i == pf::NQT - 1) tc::commit(bar(pf::B_KEMPTY + ks));
       };
       auto pv = [&](int i, int t) -> bool {  // O_i += P_i V_t
         const int vs = t % pf::VSTAGES;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_PFULL + i), t & 1))) return false;
+        if (!mbar_wait(bar(pf::B_PFULL + i), t & 1)) return false;
         if (i == 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_VFULL + vs), (t / pf::VSTAGES) & 1))) return false;
+          if (!mbar_wait(bar(pf::B_VFULL + vs), (t / pf::VSTAGES) & 1)) return false;
           if (tail_rows != 0 && tail_page / 8 == t) {
             // rows past the end of the context hold stale data that a zero
             // probability would not cancel if it were NaN: clear them
             unsigned char* vp = sbase + pf::V_OFF + vs * pf::TILE_BYTES + (tail_page % 8) * pf::PAGE_BOX_BYTES;
             const int nvec = (16 - tail_rows) * 8;  // 16-byte vectors per half
-            for (int e = lane; e < 2 * nvec; e += 32) {
+            for (int e = 0; e < 2 * nvec; ++e) {
               const int half = e / nvec, k = e % nvec;
               *reinterpret_cast<uint4*>(vp + half * pf::HALF_BYTES + tail_rows * 128 + k * 16) =
                   make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
-            __syncwarp();
           }
         }
         tc::fence_after_sync();
-        if (lane == 0) {
-          const uint64_t dv = desc_v + vs * TILE16;
-          const uint32_t p_t = tmem + i * pf::TILE_COLS;
-          const uint32_t d_o = p_t + pf::O_COL;
+        const uint64_t dv = desc_v + vs * TILE16;
+        const uint32_t p_t = tmem + i * pf::TILE_COLS;
+        const uint32_t d_o = p_t + pf::O_COL;
 #pragma unroll
-          for (int kk = 0; kk < pf::BN / 16; ++kk)
-            tc::mma_ts(d_o, p_t + kk * 8, dv + kk * (2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-          tc::commit(bar(pf::B_OREADY + i));
-          if (i == pf::NQT - 1) tc::commit(bar(pf::B_VEMPTY + vs));
-        }
-        __syncwarp();
+        for (int kk = 0; kk < pf::BN / 16; ++kk)
+          tc::mma_ts(d_o, p_t + kk * 8, dv + kk * (2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        tc::commit(bar(pf::B_OREADY + i));
+        if (i == pf::NQT - 1) tc::commit(bar(pf::B_VEMPTY + vs));
         return true;
       };
 
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(pf::B_KFULL), 0));
+      if (ok) ok = mbar_wait(bar(pf::B_KFULL), 0);
       if (ok) {
         tc::fence_after_sync();
         for (int i = 0; i < pf::NQT; ++i) qk(i, 0);
@@ -333,8 +328,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         const int ks = j % pf::KSTAGES;
         for (int i = 0; i < pf::NQT && ok; ++i) {
           ok = pv(i, j - 1);  // frees query tile i's score buffer (P_{j-1} is read first)
-          if (ok && i == 0)
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(pf::B_KFULL + ks), (j / pf::KSTAGES) & 1));
+          if (ok && i == 0) ok = mbar_wait(bar(pf::B_KFULL + ks), (j / pf::KSTAGES) & 1);
           if (ok) {
             tc::fence_after_sync();
             qk(i, j);
@@ -343,11 +337,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       }
       for (int i = 0; i < pf::NQT && ok; ++i) ok = pv(i, n_tiles - 1);
       // all MMAs of this CTA retired before TMEM is released
-      if (lane == 0) {
-        tc::commit(bar(pf::B_MMADONE));
-        mbar_wait(bar(pf::B_MMADONE), 0);
-      }
-      __syncwarp();
+      tc::commit(bar(pf::B_MMADONE));
+      mbar_wait(bar(pf::B_MMADONE), 0);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(pf::REGS_HIGH));
