@@ -463,6 +463,7 @@ pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* 
   // and the shortest fill the last one.
   const int nct = (max_q_len + ppc - 1) / ppc;
   if (nct > 65535 || B > 65535) return PKV_ERR_UNSUPPORTED;
+  p.nct = nct;
   dim3 grid(Hkv, B, nct);
   pkv::prefill_attn_kernel<<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
       p, tm_q, tm_k, tm_v);

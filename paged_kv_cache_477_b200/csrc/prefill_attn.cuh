@@ -11,9 +11,11 @@
 // it belongs on the tensor cores.
 //
 // B200 design (one CTA per SM, 12 warps):
-//   * A CTA owns two 128-row query tiles of one (sequence, kv head).  The G
-//     query heads of the kv head are packed into the rows (row = position * G
-//     + head), so every K/V tile loaded feeds 256 query rows.
+//   * A CTA owns a task: two 128-row query tiles of one (sequence, kv head).
+//     The G query heads of the kv head are packed into the rows (row =
+//     position * G + head), so every K/V tile loaded feeds 256 query rows.
+//     The last query tiles of a chunk see the most keys; they are launched
+//     first so the shortest CTAs fill the last wave.
 //   * Warp 0 (lanes 0-7) loads Q once and K/V tiles through separate K and V
 //     rings with tiled TMA: each 16-key page of the paged cache is one
 //     16 x 64-element box per head-dim half, landing in the 128-byte-swizzled
@@ -48,6 +50,7 @@ struct PrefillParams {
   const int32_t* block_tables;     // [B][MB]
   const int32_t* context_lens;     // [B]
   int32_t B, Hq, Hkv, NB, MB, G, sumQ;
+  int32_t nct;                     // tasks (query-tile pairs) per (sequence, kv head)
   float scale_log2;                // scale * log2(e), >= 0
 };
 
@@ -124,6 +127,36 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   return make_float2(__uint_as_float(__float_as_uint(p.x) + ex), __uint_as_float(__float_as_uint(p.y) + ey));
 }
 
+// Task t of a launch: query-tile pair ct of sequence b, kv head kvh, in grid
+// order (kv head fastest, then sequence, then the pairs last first).  n is
+// the number of 128-key tiles its rows see (0: nothing to do).  Each role of
+// the CTA computes it for itself (three cached loads) instead of keeping it
+// live across the register split.
+struct PrefillTask {
+  int b, kvh, ct, qs, Qb, L, p0, n;
+};
+
+__device__ __forceinline__ PrefillTask prefill_task(const PrefillParams& p, int t) {
+  PrefillTask k;
+  const int per = p.B * p.Hkv;
+  k.ct = p.nct - 1 - t / per;
+  k.b = (t % per) / p.Hkv;
+  k.kvh = t % p.Hkv;
+  k.qs = __ldg(p.query_start_loc + k.b);
+  k.Qb = __ldg(p.query_start_loc + k.b + 1) - k.qs;
+  k.L = __ldg(p.context_lens + k.b);
+  k.p0 = k.ct * pf::NQT * (pf::BM / p.G);
+  k.n = 0;
+  if (k.Qb < 0 || k.L < k.Qb || k.L > p.MB * 16 || k.qs < 0 || k.qs + k.Qb > p.sumQ) {
+    set_error(PKV_ERR_BOUNDS);
+  } else if (k.p0 < k.Qb) {
+    const int last_pos = min(k.p0 + pf::NQT * (pf::BM / p.G), k.Qb) - 1;
+    const int kv_end = k.L - k.Qb + last_pos + 1;  // keys the last valid row can see
+    k.n = (kv_end + pf::BN - 1) / pf::BN;
+  }
+  return k;
+}
+
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -132,31 +165,18 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* sbase = smem_raw + (base - raw);
 
-  const int kvh = blockIdx.x, b = blockIdx.y, ct = gridDim.z - 1 - blockIdx.z;  // last query tile first
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G, PPT = pf::BM / G;  // query positions per tile
-
-  const int qs = __ldg(p.query_start_loc + b);
-  const int Qb = __ldg(p.query_start_loc + b + 1) - qs;
-  const int L = __ldg(p.context_lens + b);
-  const int p0 = ct * pf::NQT * PPT;      // first position of query tile 0
+  const int t = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;  // this CTA's task
 
   __shared__ int s_flag;
   if (threadIdx.x == 0) {
     int f = *reinterpret_cast<volatile int*>(&g_error_word) == PKV_ERR_TIMEOUT;
-    if (Qb < 0 || L < Qb || L > p.MB * 16 || qs < 0 || qs + Qb > p.sumQ) {
-      set_error(PKV_ERR_BOUNDS);
-      f = 1;
-    }
+    f |= prefill_task(p, t).n == 0;  // nothing to do (or bad lengths, reported)
     s_flag = f;
   }
   __syncthreads();
-  if (s_flag || p0 >= Qb) return;
-
-  const int last_pos = min(p0 + pf::NQT * PPT, Qb) - 1;
-  const int kv_end = L - Qb + last_pos + 1;  // keys the last valid row can see
-  const int n_tiles = (kv_end + pf::BN - 1) / pf::BN;
-  const int npages = (L + 15) / 16;
+  if (s_flag) return;
 
   auto bar = [&](int i) { return base + pf::BAR_OFF + 8u * i; };
   if (threadIdx.x == 0) {
@@ -198,17 +218,22 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         tc::prefetch_tensormap(&tm_q);
         tc::prefetch_tensormap(&tm_k);
         tc::prefetch_tensormap(&tm_v);
+      }
+      const PrefillTask k = prefill_task(p, t);
+      if (lane == 0) {
         mbar_arrive_expect_tx(bar(pf::B_Q), pf::NQT * pf::TILE_BYTES);
         for (int i = 0; i < pf::NQT; ++i) {
           const uint32_t qd = base + pf::Q_OFF + i * pf::TILE_BYTES;
-          const int z = qs + p0 + i * PPT;
-          tc::tma_load_3d(qd, &tm_q, 0, kvh * G, z, bar(pf::B_Q));
-          tc::tma_load_3d(qd + pf::HALF_BYTES, &tm_q, 64, kvh * G, z, bar(pf::B_Q));
+          const int z = k.qs + k.p0 + i * PPT;
+          tc::tma_load_3d(qd, &tm_q, 0, k.kvh * G, z, bar(pf::B_Q));
+          tc::tma_load_3d(qd + pf::HALF_BYTES, &tm_q, 64, k.kvh * G, z, bar(pf::B_Q));
         }
       }
-      const int32_t* bt = p.block_tables + (size_t)b * p.MB;
+      const int32_t* bt = p.block_tables + (size_t)k.b * p.MB;
+      const int npages = (k.L + 15) / 16;
       int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < n_tiles; ++j) {
+      bool ok = true;
+      for (int j = 0; j < k.n; ++j) {
         int blk = p.NB;  // out of range: TMA fills the page with zeros
         if (lane < 8) {
           const int pg = j * 8 + lane;
@@ -222,7 +247,6 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         }
         // K tile j
         const int ks = j % pf::KSTAGES;
-        bool ok = true;
         if (lane == 0) {
           if (j >= pf::KSTAGES) ok = mbar_wait(bar(pf::B_KEMPTY + ks), ((j / pf::KSTAGES) - 1) & 1);
           if (ok) mbar_arrive_expect_tx(bar(pf::B_KFULL + ks), pf::TILE_BYTES);
@@ -230,8 +254,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         if (lane < 8) {
           const uint32_t kd = base + pf::K_OFF + ks * pf::TILE_BYTES + lane * pf::PAGE_BOX_BYTES;
-          tc::tma_load_4d(kd, &tm_k, 0, 0, kvh, blk, bar(pf::B_KFULL + ks));
-          tc::tma_load_4d(kd + pf::HALF_BYTES, &tm_k, 64, 0, kvh, blk, bar(pf::B_KFULL + ks));
+          tc::tma_load_4d(kd, &tm_k, 0, 0, k.kvh, blk, bar(pf::B_KFULL + ks));
+          tc::tma_load_4d(kd + pf::HALF_BYTES, &tm_k, 64, 0, k.kvh, blk, bar(pf::B_KFULL + ks));
         }
         ++issued_k;
         // V tile j
@@ -243,12 +267,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         if (lane < 8) {
           const uint32_t vd = base + pf::V_OFF + vs * pf::TILE_BYTES + lane * pf::PAGE_BOX_BYTES;
-          tc::tma_load_4d(vd, &tm_v, 0, 0, kvh, blk, bar(pf::B_VFULL + vs));
-          tc::tma_load_4d(vd + pf::HALF_BYTES, &tm_v, 64, 0, kvh, blk, bar(pf::B_VFULL + vs));
+          tc::tma_load_4d(vd, &tm_v, 0, 0, k.kvh, blk, bar(pf::B_VFULL + vs));
+          tc::tma_load_4d(vd + pf::HALF_BYTES, &tm_v, 64, 0, k.kvh, blk, bar(pf::B_VFULL + vs));
         }
         ++issued_v;
       }
-      // leave no copy in flight: wait for the last issued use of every stage
+      // leave no copy in flight: wait for the last issued use of every buffer
       if (lane == 0) {
         mbar_wait(bar(pf::B_Q), 0);
         for (int s = 0; s < pf::KSTAGES && s < issued_k; ++s) {
@@ -266,19 +290,15 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       // MMA and commit, so no warp-wide vote sits between two MMA groups.
       constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(pf::BM, pf::BN, false, false);
       constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(pf::BM, pf::D, false, true);
-      bool ok = mbar_wait(bar(pf::B_Q), 0);
-      // the page holding the sequence's last key, if it is only partly valid
-      const int tail_rows = L % 16;
-      const int tail_page = (L - 1) / 16;
-
       // Descriptors are built once; a K step only moves the start address,
       // whose 14-bit field (address >> 4) cannot carry: shared memory < 256 KB.
       const uint64_t desc_q = tc::smem_desc_sw128(base + pf::Q_OFF, 16, 1024);
       const uint64_t desc_k = tc::smem_desc_sw128(base + pf::K_OFF, 16, 1024);
       const uint64_t desc_v = tc::smem_desc_sw128(base + pf::V_OFF, pf::HALF_BYTES, 1024);
       constexpr uint32_t TILE16 = pf::TILE_BYTES >> 4;
-      auto qk = [&](int i, int j) {  // S_i = Q_i K_j^T
-        const int ks = j % pf::KSTAGES;
+      int tk = 0, tv = 0;  // K and V tiles consumed: ring stage and phase
+      auto qk = [&](int i) {  // S_i = Q_i K^T for K tile tk
+        const int ks = tk % pf::KSTAGES;
         const uint64_t dq = desc_q + i * TILE16, dk = desc_k + ks * TILE16;
         const uint32_t d_s = tmem + i * pf::TILE_COLS;
 #pragma unroll
@@ -289,12 +309,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         tc::commit(bar(pf::B_SFULL + i));
         if (i == pf::NQT - 1) tc::commit(bar(pf::B_KEMPTY + ks));
       };
-      auto pv = [&](int i, int t) -> bool {  // O_i += P_i V_t
-        const int vs = t % pf::VSTAGES;
-        if (!mbar_wait(bar(pf::B_PFULL + i), t & 1)) return false;
+      // O_i += P_i V for V tile tv = key tile j
+      auto pv = [&](int i, int j, int tail_rows, int tail_page) -> bool {
+        const int vs = tv % pf::VSTAGES;
+        if (!mbar_wait(bar(pf::B_PFULL + i), j & 1)) return false;
         if (i == 0) {
-          if (!mbar_wait(bar(pf::B_VFULL + vs), (t / pf::VSTAGES) & 1)) return false;
-          if (tail_rows != 0 && tail_page / 8 == t) {
+          if (!mbar_wait(bar(pf::B_VFULL + vs), (tv / pf::VSTAGES) & 1)) return false;
+          if (tail_rows != 0 && tail_page / 8 == j) {
             // rows past the end of the context hold stale data that a zero
             // probability would not cancel if it were NaN: clear them
             unsigned char* vp = sbase + pf::V_OFF + vs * pf::TILE_BYTES + (tail_page % 8) * pf::PAGE_BOX_BYTES;
@@ -313,29 +334,37 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         const uint32_t d_o = p_t + pf::O_COL;
 #pragma unroll
         for (int kk = 0; kk < pf::BN / 16; ++kk)
-          tc::mma_ts(d_o, p_t + kk * 8, dv + kk * (2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(d_o, p_t + kk * 8, dv + kk * (2048 >> 4), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         tc::commit(bar(pf::B_OREADY + i));
-        if (i == pf::NQT - 1) tc::commit(bar(pf::B_VEMPTY + vs));
+        if (i == pf::NQT - 1) {
+          tc::commit(bar(pf::B_VEMPTY + vs));
+          ++tv;
+        }
         return true;
       };
 
+      const PrefillTask k = prefill_task(p, t);
+      // the page holding the sequence's last key, if it is only partly valid
+      const int tail_rows = k.L % 16, tail_page = (k.L - 1) / 16;
+      bool ok = mbar_wait(bar(pf::B_Q), 0);
       if (ok) ok = mbar_wait(bar(pf::B_KFULL), 0);
       if (ok) {
         tc::fence_after_sync();
-        for (int i = 0; i < pf::NQT; ++i) qk(i, 0);
+        for (int i = 0; i < pf::NQT; ++i) qk(i);
+        ++tk;
       }
-      for (int j = 1; j < n_tiles && ok; ++j) {
-        const int ks = j % pf::KSTAGES;
+      for (int j = 1; j < k.n && ok; ++j) {
         for (int i = 0; i < pf::NQT && ok; ++i) {
-          ok = pv(i, j - 1);  // frees query tile i's score buffer (P_{j-1} is read first)
-          if (ok && i == 0) ok = mbar_wait(bar(pf::B_KFULL + ks), (j / pf::KSTAGES) & 1);
+          ok = pv(i, j - 1, tail_rows, tail_page);  // frees query tile i's score buffer (P_{j-1} is read first)
+          if (ok && i == 0) ok = mbar_wait(bar(pf::B_KFULL + tk % pf::KSTAGES), (tk / pf::KSTAGES) & 1);
           if (ok) {
             tc::fence_after_sync();
-            qk(i, j);
+            qk(i);
           }
         }
+        ++tk;
       }
-      for (int i = 0; i < pf::NQT && ok; ++i) ok = pv(i, n_tiles - 1);
+      for (int i = 0; i < pf::NQT && ok; ++i) ok = pv(i, k.n - 1, tail_rows, tail_page);
       // all MMAs of this CTA retired before TMEM is released
       tc::commit(bar(pf::B_MMADONE));
       mbar_wait(bar(pf::B_MMADONE), 0);
@@ -346,126 +375,130 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     const int qt = (warp - 4) >> 2;              // query tile of this warpgroup
     const int wq = warp & 3;                     // TMEM lane quarter of this warp
     const int r = wq * 32 + lane;                // row within the query tile
-    const int pos = p0 + qt * PPT + r / G, hh = r % G;
-    const bool row_valid = pos < Qb;
-    const int limit = L - Qb + min(pos, Qb - 1);  // last key this row may see
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t s_addr = tmem + lane_off + qt * pf::TILE_COLS;
     const uint32_t o_addr = s_addr + pf::O_COL;
     const float sl2 = p.scale_log2;
+    const PrefillTask k = prefill_task(p, t);
+    const int pos = k.p0 + qt * PPT + r / G, hh = r % G;
+    const bool row_valid = pos < k.Qb;
+    const int limit = k.L - k.Qb + min(pos, k.Qb - 1);  // last key this row may see
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_SFULL + qt), j & 1))) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
-      uint32_t sr[pf::BN];
-#pragma unroll
-      for (int c = 0; c < pf::BN; c += 32) tc::ld_32x32b_x32(s_addr + c, sr + c);
-      tc::wait_ld();
-      const int kv0 = j * pf::BN;
-      const bool diag = kv0 + pf::BN - 1 > limit;
-      if (diag) {
-#pragma unroll
-        for (int c = 0; c < pf::BN; ++c)
-          if (kv0 + c > limit) sr[c] = __float_as_uint(-INFINITY);
-      }
-      // row max: eight independent chains of three-input maxima
-      float mxk[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        float m = fmax3(__uint_as_float(sr[16 * k]), __uint_as_float(sr[16 * k + 1]),
-                        __uint_as_float(sr[16 * k + 2]));
-#pragma unroll
-        for (int e = 3; e < 15; e += 2)
-          m = fmax3(m, __uint_as_float(sr[16 * k + e]), __uint_as_float(sr[16 * k + e + 1]));
-        mxk[k] = fmaxf(m, __uint_as_float(sr[16 * k + 15]));
-      }
-      const float mx = fmax3(fmax3(mxk[0], mxk[1], mxk[2]), fmax3(mxk[3], mxk[4], mxk[5]), fmaxf(mxk[6], mxk[7]));
-      const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sl2;
-      const bool grow = m_tile > m_run + pf::RESCALE_THRESHOLD;  // always true on the first tile
-      if (__any_sync(0xffffffffu, grow)) {
-        // warp-uniform branch: the TMEM accesses below are warp-collective;
-        // rows that keep their max use alpha = 1
-        const float alpha = grow ? ex2(m_run - m_tile) : 1.f;  // 0 on the first tile
-        if (j > 0) {
-          // O holds P.V of earlier tiles: rescale it once the last of them is done
-          if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (j - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          tc::fence_after_sync();
-#pragma unroll
-          for (int c = 0; c < pf::D; c += 32) {
-            uint32_t o[32];
-            tc::ld_32x32b_x32(o_addr + c, o);
-            tc::wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tc::st_32x32b_x32(o_addr + c, o);
-          }
-          tc::wait_st();
+    {  // key tiles, then the epilogue
+      for (int j = 0; j < k.n; ++j) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_SFULL + qt), j & 1))) {
+          ok = false;
+          break;
         }
-        if (grow) {
-          l_run *= alpha;
-          m_run = m_tile;
-        }
-      }
-      // P = 2^(s * scale_log2 - m) as bf16 pairs, written over the score
-      // columns in two halves so the first store overlaps the second half
-      const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_run, -m_run);
-      float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                      make_float2(0.f, 0.f)};
-      uint32_t* pw = sr;  // packed P overwrites the scores already consumed (c/2 < c)
+        tc::fence_after_sync();
+        uint32_t sr[pf::BN];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-#pragma unroll
-        for (int c = half * 64; c < half * 64 + 64; c += 2) {
-          const float2 x =
-              __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
-          float2 pr = pf::poly_pair(c / 2)
-                          ? exp2_poly2(x)
-                          : make_float2(ex2(x.x), ex2(x.y));
-          if (diag) {  // masked keys: exactly 0 (the polynomial, or a zero scale, would not give it)
-            if (kv0 + c > limit) pr.x = 0.f;
-            if (kv0 + c + 1 > limit) pr.y = 0.f;
-          }
-          rs[(c / 2) & 3] = __fadd2_rn(rs[(c / 2) & 3], pr);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(pr.x, pr.y);
-          pw[c / 2] = *reinterpret_cast<uint32_t*>(&h2);
-        }
-        tc::st_32x32b_x32(s_addr + half * 32, pw + half * 32);
-      }
-      const float2 r01 = __fadd2_rn(rs[0], rs[1]), r23 = __fadd2_rn(rs[2], rs[3]);
-      const float2 r = __fadd2_rn(r01, r23);
-      l_run += r.x + r.y;
-      tc::wait_st();
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(pf::B_PFULL + qt));
-    }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (n_tiles - 1) & 1))) {
-      tc::fence_after_sync();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)(qs + pos) * p.Hq + kvh * G + hh) * pf::D);
-#pragma unroll
-      for (int c = 0; c < pf::D; c += 32) {
-        uint32_t o[32];
-        tc::ld_32x32b_x32(o_addr + c, o);
+        for (int c = 0; c < pf::BN; c += 32) tc::ld_32x32b_x32(s_addr + c, sr + c);
         tc::wait_ld();
-        if (row_valid) {
+        const int kv0 = j * pf::BN;
+        const bool diag = kv0 + pf::BN - 1 > limit;
+        if (diag) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t w[4];
+          for (int c = 0; c < pf::BN; ++c)
+            if (kv0 + c > limit) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // row max: eight independent chains of three-input maxima
+        float mxk[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[v * 8 + 2 * e]) * inv,
-                                                        __uint_as_float(o[v * 8 + 2 * e + 1]) * inv);
-              w[e] = *reinterpret_cast<uint32_t*>(&h2);
+        for (int k = 0; k < 8; ++k) {
+          float m = fmax3(__uint_as_float(sr[16 * k]), __uint_as_float(sr[16 * k + 1]),
+                          __uint_as_float(sr[16 * k + 2]));
+#pragma unroll
+          for (int e = 3; e < 15; e += 2)
+            m = fmax3(m, __uint_as_float(sr[16 * k + e]), __uint_as_float(sr[16 * k + e + 1]));
+          mxk[k] = fmaxf(m, __uint_as_float(sr[16 * k + 15]));
+        }
+        const float mx = fmax3(fmax3(mxk[0], mxk[1], mxk[2]), fmax3(mxk[3], mxk[4], mxk[5]), fmaxf(mxk[6], mxk[7]));
+        const float m_tile = (mx == -INFINITY) ? -INFINITY : mx * sl2;
+        const bool grow = m_tile > m_run + pf::RESCALE_THRESHOLD;  // always true on the first tile
+        if (__any_sync(0xffffffffu, grow)) {
+          // warp-uniform branch: the TMEM accesses below are warp-collective;
+          // rows that keep their max use alpha = 1
+          const float alpha = grow ? ex2(m_run - m_tile) : 1.f;  // 0 on the first tile
+          if (j > 0) {
+            // O holds P.V of earlier tiles: rescale it once the last of them is done
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (j - 1) & 1))) {
+              ok = false;
+              break;
             }
-            dst[c / 8 + v] = make_uint4(w[0], w[1], w[2], w[3]);
+            tc::fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < pf::D; c += 32) {
+              uint32_t o[32];
+              tc::ld_32x32b_x32(o_addr + c, o);
+              tc::wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tc::st_32x32b_x32(o_addr + c, o);
+            }
+            tc::wait_st();
+          }
+          if (grow) {
+            l_run *= alpha;
+            m_run = m_tile;
+          }
+        }
+        // P = 2^(s * scale_log2 - m) as bf16 pairs, written over the score
+        // columns in two halves so the first store overlaps the second half
+        const float2 sl2x2 = make_float2(sl2, sl2), negm = make_float2(-m_run, -m_run);
+        float2 rs[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        uint32_t* pw = sr;  // packed P overwrites the scores already consumed (c/2 < c)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int c = half * 64; c < half * 64 + 64; c += 2) {
+            const float2 x =
+                __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
+            float2 pr = pf::poly_pair(c / 2)
+                            ? exp2_poly2(x)
+                            : make_float2(ex2(x.x), ex2(x.y));
+            if (diag) {  // masked keys: exactly 0 (the polynomial, or a zero scale, would not give it)
+              if (kv0 + c > limit) pr.x = 0.f;
+              if (kv0 + c + 1 > limit) pr.y = 0.f;
+            }
+            rs[(c / 2) & 3] = __fadd2_rn(rs[(c / 2) & 3], pr);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(pr.x, pr.y);
+            pw[c / 2] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          tc::st_32x32b_x32(s_addr + half * 32, pw + half * 32);
+        }
+        const float2 r01 = __fadd2_rn(rs[0], rs[1]), r23 = __fadd2_rn(rs[2], rs[3]);
+        const float2 rr = __fadd2_rn(r01, r23);
+        l_run += rr.x + rr.y;
+        tc::wait_st();
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(pf::B_PFULL + qt));
+      }
+      if (ok && __all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (k.n - 1) & 1))) {
+        tc::fence_after_sync();
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)(k.qs + pos) * p.Hq + k.kvh * G + hh) * pf::D);
+        // O / l to global memory
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+        for (int c = 0; c < pf::D; c += 32) {
+          uint32_t o[32];
+          tc::ld_32x32b_x32(o_addr + c, o);
+          tc::wait_ld();
+          if (row_valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[v * 8 + 2 * e]) * inv,
+                                                          __uint_as_float(o[v * 8 + 2 * e + 1]) * inv);
+                w[e] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              dst[c / 8 + v] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
       }
