@@ -80,8 +80,13 @@ class Oracle:
         lib.ref_paged_attention_prefill.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32]
         lib.ref_decode_partials.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32, _I32, _I32]
         lib.ref_lse_merge.argtypes = [_P, _P, _P, _I64, _I32, _I32]
+        lib.ref_kv_cache_write_int8.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I32, _I32, _I32,
+                                                _I32, _I32]
+        lib.ref_paged_attention_int8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32,
+                                                 _I32, _I32, _F32]
         for f in ("ref_kv_cache_write", "ref_paged_attention", "ref_contiguous_attention",
-                  "ref_paged_attention_prefill", "ref_decode_partials", "ref_lse_merge"):
+                  "ref_paged_attention_prefill", "ref_decode_partials", "ref_lse_merge",
+                  "ref_kv_cache_write_int8", "ref_paged_attention_int8"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
         self.mutant = lib.ref_mutant_id()
@@ -108,6 +113,38 @@ class Oracle:
         rc = self.lib.ref_kv_cache_write(_ptr(key), _ptr(value), Hkv * D, Hkv * D, _ptr(k_cache),
                                          _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D, NB, bs)
         return self._check(rc, "kv_cache_write", allow_bounds)
+
+    def kv_cache_write_int8(self, key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping,
+                            allow_bounds=False) -> int:
+        """Quantise key/value [T, Hkv, D] (uint16 bf16 bits) into the int8 pools
+        k_cache/v_cache [NB, Hkv, bs, D] and their fp32 scales [NB, Hkv, bs], in place."""
+        T, Hkv, D = key.shape
+        NB, Hkv2, bs, D2 = k_cache.shape
+        assert Hkv == Hkv2 and D == D2 and value.shape == key.shape and v_cache.shape == k_cache.shape
+        assert k_cache.dtype == np.int8 and k_scale.dtype == np.float32 and k_scale.shape == (NB, Hkv, bs)
+        slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        key = np.ascontiguousarray(key)
+        value = np.ascontiguousarray(value)
+        rc = self.lib.ref_kv_cache_write_int8(_ptr(key), _ptr(value), Hkv * D, Hkv * D, _ptr(k_cache),
+                                              _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping),
+                                              T, Hkv, D, NB, bs)
+        return self._check(rc, "kv_cache_write_int8", allow_bounds)
+
+    def paged_attention_int8(self, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
+                             allow_bounds=False) -> np.ndarray:
+        """Decode over the int8 pools: attention over the values code * scale."""
+        B, Hq, D = q.shape
+        NB, Hkv, bs, _ = k_cache.shape
+        assert k_cache.dtype == np.int8 and k_scale.dtype == np.float32
+        block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+        context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+        MB = block_tables.shape[1] if block_tables.ndim == 2 else 0
+        out = np.zeros((B, Hq, D), dtype=np.float64)
+        rc = self.lib.ref_paged_attention_int8(_ptr(out), _ptr(np.ascontiguousarray(q)), _ptr(k_cache),
+                                               _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+                                               MB, _ptr(context_lens), B, Hq, Hkv, D, NB, bs, float(scale))
+        self._check(rc, "paged_attention_int8", allow_bounds)
+        return out
 
     # -- decode ----------------------------------------------------------------
     def paged_attention(self, q, k_cache, v_cache, block_tables, context_lens, scale,

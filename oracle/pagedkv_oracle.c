@@ -421,3 +421,173 @@ int ref_lse_merge(double* out, const double* o_part, const double* lse,
   }
   return ORC_OK;
 }
+
+/* ========================================================================= */
+/* INT8 KV cache with one fp32 scale per (token, kv head).                    */
+/*                                                                            */
+/* The pages name an INT8 KV cache as the way to halve its memory            */
+/* (Tiny-Infer page, section "推测性解码与INT8量化"); they fix neither the     */
+/* scale granularity nor the rounding.  Reading taken here: symmetric, one    */
+/* scale per written row (a token's D values of one kv head), the only        */
+/* granularity an incremental cache write can fix when the row is written;    */
+/*   amax = max_d |x_d|;  scale = amax / 127;  inv = 127 / amax;              */
+/*   code_d = clamp(round_half_even(x_d * inv), -127, 127);                   */
+/* all in fp32 (x is bf16 widened exactly), so the codes are one exact        */
+/* function of the row; amax = 0 gives codes 0 and scale 0.  The row's value  */
+/* is code_d * scale, exact in fp64, and attention is the plain definition    */
+/* over those values.                                                         */
+/* Pools: k_cache/v_cache int8 [NB][Hkv][bs][D]; k_scale/v_scale fp32         */
+/* [NB][Hkv][bs].                                                             */
+/* ========================================================================= */
+
+static float bf16_bits_to_f32(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* quantise one row of D bf16 values */
+static void quantize_row_int8(int8_t* codes, float* scale_out, const uint16_t* x, int32_t D) {
+  float amax = 0.0f;
+  for (int32_t d = 0; d < D; ++d) {
+    const float a = fabsf(bf16_bits_to_f32(x[d]));
+    if (a > amax) amax = a;
+  }
+  if (amax == 0.0f) {
+    for (int32_t d = 0; d < D; ++d) codes[d] = 0;
+    *scale_out = 0.0f;
+    return;
+  }
+#if PKV_ORACLE_MUTANT == 11
+  const float inv = 128.0f / amax; /* planted: wrong code range */
+#else
+  const float inv = 127.0f / amax;
+#endif
+  for (int32_t d = 0; d < D; ++d) {
+    const float y = bf16_bits_to_f32(x[d]) * inv;
+#if PKV_ORACLE_MUTANT == 12
+    float r = truncf(y); /* planted: rounds toward zero */
+#else
+    float r = rintf(y); /* round half to even (default rounding mode) */
+#endif
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    codes[d] = (int8_t)r;
+  }
+  *scale_out = amax / 127.0f;
+}
+
+/* Quantise new K/V rows into their slots (see ref_kv_cache_write for the
+ * scatter itself).  key/value [T][Hkv][D] bf16 bits, token stride in
+ * elements. */
+int ref_kv_cache_write_int8(const uint16_t* key, const uint16_t* value,
+                            int64_t key_stride_tok, int64_t value_stride_tok,
+                            int8_t* k_cache, int8_t* v_cache, float* k_scale,
+                            float* v_scale, const int64_t* slot_mapping,
+                            int32_t T, int32_t Hkv, int32_t D, int32_t NB,
+                            int32_t bs) {
+  if (T < 0 || Hkv <= 0 || D <= 0 || NB < 0 || bs <= 0) return ORC_INVALID;
+  const int64_t pool_slots = (int64_t)NB * bs;
+  int status = ORC_OK;
+  for (int64_t t = 0; t < T; ++t) {
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= pool_slots) {
+      status = ORC_BOUNDS;
+      continue;
+    }
+    const int64_t blk = slot / bs, off = slot % bs;
+    for (int32_t h = 0; h < Hkv; ++h) {
+      const int64_t row = (blk * Hkv + h) * bs + off;
+      quantize_row_int8(k_cache + row * D, k_scale + row, key + t * key_stride_tok + (int64_t)h * D, D);
+      quantize_row_int8(v_cache + row * D, v_scale + row, value + t * value_stride_tok + (int64_t)h * D, D);
+    }
+  }
+  return status;
+}
+
+/* Attention of one query row over n int8 rows with their scales; same two
+ * passes as attend_row. */
+static void attend_row_int8(double* out, const double* q, int32_t D, double scale,
+                            const int8_t* const* krows, const float* ks,
+                            const int8_t* const* vrows, const float* vs, int64_t n,
+                            double* s) {
+  for (int32_t d = 0; d < D; ++d) out[d] = 0.0;
+  if (n <= 0) return;
+  double m = -INFINITY;
+  for (int64_t j = 0; j < n; ++j) {
+    double dot = 0.0;
+    for (int32_t d = 0; d < D; ++d) dot += q[d] * ((double)krows[j][d] * (double)ks[j]);
+    s[j] = scale * dot;
+    if (s[j] > m) m = s[j];
+  }
+  double l = 0.0;
+  for (int64_t j = 0; j < n; ++j) {
+    s[j] = exp(s[j] - m);
+    l += s[j];
+  }
+  for (int64_t j = 0; j < n; ++j) {
+#if PKV_ORACLE_MUTANT == 13
+    const double vscale = (double)ks[j]; /* planted: V rows scaled by the K scale */
+#else
+    const double vscale = (double)vs[j];
+#endif
+    for (int32_t d = 0; d < D; ++d) out[d] += s[j] * ((double)vrows[j][d] * vscale);
+  }
+  for (int32_t d = 0; d < D; ++d) out[d] /= l;
+}
+
+/* Decode over the int8 pool; same gather and grouped-query mapping as
+ * ref_paged_attention. */
+int ref_paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cache,
+                             const int8_t* v_cache, const float* k_scale,
+                             const float* v_scale, const int32_t* block_tables,
+                             int32_t MB, const int32_t* context_lens, int32_t B,
+                             int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                             int32_t bs, float scale) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || MB < 0 ||
+      Hq % Hkv != 0)
+    return ORC_INVALID;
+  for (int32_t b = 0; b < B; ++b)
+    if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)MB * bs)
+      return ORC_INVALID;
+  int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < (int64_t)B * Hq; ++bh) {
+    const int32_t b = (int32_t)(bh / Hq), h = (int32_t)(bh % Hq);
+    const int64_t n = context_lens[b];
+    const int32_t g = kv_head_of(h, Hq, Hkv);
+    const int8_t** kr = (const int8_t**)malloc(sizeof(void*) * (n + 1));
+    const int8_t** vr = (const int8_t**)malloc(sizeof(void*) * (n + 1));
+    float* ks = (float*)malloc(sizeof(float) * (n + 1));
+    float* vs = (float*)malloc(sizeof(float) * (n + 1));
+    double* s = (double*)malloc(sizeof(double) * (n + 1));
+    double* qd = (double*)malloc(sizeof(double) * D);
+    int bad = 0;
+    for (int64_t j = 0; j < n; ++j) {
+      const int64_t page = j / bs, row = j % bs;
+      const int32_t blk = block_tables[(int64_t)b * MB + page];
+      if (blk < 0 || blk >= NB) {
+        bad = 1;
+        break;
+      }
+      const int64_t r = ((int64_t)blk * Hkv + g) * bs + row;
+      kr[j] = k_cache + r * D;
+      vr[j] = v_cache + r * D;
+      ks[j] = k_scale[r];
+      vs[j] = v_scale[r];
+    }
+    double* o = out + bh * D;
+    if (bad) {
+      for (int32_t d = 0; d < D; ++d) o[d] = NAN;
+#pragma omp atomic write
+      status = ORC_BOUNDS;
+    } else {
+      widen_row(qd, q + bh * D, D);
+      attend_row_int8(o, qd, D, (double)scale, kr, ks, vr, vs, n, s);
+    }
+    free(kr); free(vr); free(ks); free(vs); free(s); free(qd);
+  }
+  return status;
+}

@@ -22,7 +22,13 @@ section "分页KV缓存：借鉴操作系统的内存管理"; exact softmax atte
 * causal: future keys do not matter; the last query of a chunk equals decode;
 * GQA equals materialised MHA; G = 1 is plain MHA;
 * split-KV partials merged by log-sum-exp equal the plain result;
-* an empty context gives a zero row.
+* an empty context gives a zero row;
+* INT8 cache (one fp32 scale per token row, the reading of the Tiny-Infer
+  page's section "推测性解码与INT8量化"): rows built as k * 2^-e decode to
+  exactly k and 2^-e; ties round to even; every value is within scale/2 of
+  its code; a zero row gives zero codes and scale; attention over the int8
+  pool equals NumPy brute force over the dequantised values, and equals the
+  pinned bf16 path bit for bit when the values are bf16-exact.
 """
 from __future__ import annotations
 
@@ -322,6 +328,146 @@ def pin_empty_context_is_zero(orc):
     assert np.isfinite(out[1]).all()
 
 
+# --------------------------------------------------------------------------- #
+# INT8 cache                                                                   #
+# --------------------------------------------------------------------------- #
+
+def _int8_pool(NB, Hkv, bs, D):
+    """Empty int8 pools with canaries: code 99 and a NaN scale in every slot."""
+    k = np.full((NB, Hkv, bs, D), 99, dtype=np.int8)
+    v = np.full((NB, Hkv, bs, D), 99, dtype=np.int8)
+    ks = np.full((NB, Hkv, bs), np.nan, dtype=np.float32)
+    vs = np.full((NB, Hkv, bs), np.nan, dtype=np.float32)
+    return k, v, ks, vs
+
+
+def pin_int8_exact_grid_rows(orc):
+    """Values k * 2^-e with max |k| = 127 are bf16-exact; the row's scale is
+    then exactly 2^-e and its codes exactly k."""
+    rng = np.random.default_rng(31)
+    T, Hkv, D, bs, NB = 6, 2, 32, 4, 3
+    kk = rng.integers(-127, 128, size=(T, Hkv, D))
+    kk[..., 0] = 127 * np.where(rng.random((T, Hkv)) < 0.5, 1, -1)   # amax = 127 * 2^-e
+    e = rng.integers(0, 12, size=(T, Hkv, 1))
+    x = (kk * np.ldexp(1.0, -e)).astype(np.float32)
+    bits = f32_to_bf16_bits(x)
+    assert np.array_equal(bf16_bits_to_f64(bits), x.astype(np.float64))
+    k, v, ks, vs = _int8_pool(NB, Hkv, bs, D)
+    slots = np.array([0, 5, 2, 11, 7, 3], dtype=np.int64)
+    orc.kv_cache_write_int8(bits, bits, k, v, ks, vs, slots)
+    for t, sl in enumerate(slots):
+        blk, off = sl // bs, sl % bs
+        assert np.array_equal(k[blk, :, off, :], kk[t].astype(np.int8))
+        assert np.array_equal(v[blk, :, off, :], kk[t].astype(np.int8))
+        assert np.array_equal(ks[blk, :, off], np.ldexp(1.0, -e[t, :, 0]).astype(np.float32))
+
+
+def pin_int8_ties_round_to_even(orc):
+    """amax = 127 makes the code step exactly 1: x.5 rounds to the even code."""
+    row = np.array([127.0, 2.5, 3.5, -2.5, -0.5, 0.5, 1.5, -1.5, 126.5, 0.25, -3.5, 4.5], dtype=np.float32)
+    want = np.array([127, 2, 4, -2, 0, 0, 2, -2, 126, 0, -4, 4], dtype=np.int8)
+    bits = f32_to_bf16_bits(row)[None, None, :]
+    k, v, ks, vs = _int8_pool(1, 1, 1, row.size)
+    orc.kv_cache_write_int8(bits, bits, k, v, ks, vs, np.array([0], dtype=np.int64))
+    assert np.array_equal(k[0, 0, 0], want), k[0, 0, 0]
+    assert ks[0, 0, 0] == np.float32(1.0)
+
+
+def pin_int8_error_within_half_step(orc):
+    """Round to nearest: |code * scale - x| <= scale / 2, every code in
+    [-127, 127], and the largest |code| is 127.  Slack: x * inv and the stored
+    scale are fp32, each off by <= 2^-24 relative, i.e. <= 127 * 2^-23 of a
+    code step near a tie; 2^-14 of the half step covers it, far below the
+    whole step a truncating rounding would miss by."""
+    rng = np.random.default_rng(32)
+    T, Hkv, D, bs, NB = 40, 3, 64, 8, 6
+    bits = rand_bits(rng, (T, Hkv, D), std=2.0)
+    k, v, ks, vs = _int8_pool(NB, Hkv, bs, D)
+    slots = rng.permutation(NB * bs)[:T].astype(np.int64)
+    orc.kv_cache_write_int8(bits, bits, k, v, ks, vs, slots)
+    x = bf16_bits_to_f64(bits)
+    for t, sl in enumerate(slots):
+        blk, off = sl // bs, sl % bs
+        c = k[blk, :, off, :].astype(np.float64)
+        sc = ks[blk, :, off].astype(np.float64)[:, None]
+        assert np.abs(c).max() <= 127
+        assert np.all(np.abs(c).max(axis=-1) == 127)
+        assert np.all(np.abs(c * sc - x[t]) <= 0.5 * sc * (1 + 2.0 ** -14))
+
+
+def pin_int8_zero_row_and_slots(orc):
+    """A zero row gives codes 0 and scale 0; negative slots are skipped and
+    every other slot keeps its canary."""
+    D, bs, NB = 16, 4, 2
+    key = np.zeros((3, 1, D), dtype=np.uint16)
+    key[1] = f32_to_bf16_bits(np.linspace(-1, 1, D, dtype=np.float32))[None]
+    k, v, ks, vs = _int8_pool(NB, 1, bs, D)
+    orc.kv_cache_write_int8(key, key, k, v, ks, vs, np.array([6, -1, 1], dtype=np.int64))
+    assert np.array_equal(k[1, 0, 2], np.zeros(D, np.int8)) and ks[1, 0, 2] == 0.0
+    assert np.array_equal(k[0, 0, 1], np.zeros(D, np.int8)) and ks[0, 0, 1] == 0.0
+    touched = {(1, 2), (0, 1)}
+    for blk in range(NB):
+        for off in range(bs):
+            if (blk, off) not in touched:
+                assert np.all(k[blk, 0, off] == 99) and np.isnan(ks[blk, 0, off])
+
+
+def _random_int8_paged(rng, lens, Hkv, D, bs, extra=2):
+    pages = [-(-L // bs) for L in lens]
+    NB = sum(pages) + extra
+    perm = rng.permutation(NB)
+    MB = max(pages + [1])
+    bt = np.full((len(lens), MB), -1, dtype=np.int32)
+    o = 0
+    for b, n in enumerate(pages):
+        bt[b, :n] = perm[o:o + n]
+        o += n
+    k = rng.integers(-127, 128, size=(NB, Hkv, bs, D)).astype(np.int8)
+    v = rng.integers(-127, 128, size=(NB, Hkv, bs, D)).astype(np.int8)
+    ks = np.exp(rng.uniform(np.log(1e-3), np.log(3e-2), size=(NB, Hkv, bs))).astype(np.float32)
+    vs = np.exp(rng.uniform(np.log(1e-3), np.log(3e-2), size=(NB, Hkv, bs))).astype(np.float32)
+    return k, v, ks, vs, bt, np.array(lens, dtype=np.int32)
+
+
+def pin_int8_attention_brute_force(orc):
+    """NumPy full-matrix attention over the dequantised pool (code * scale)."""
+    rng = np.random.default_rng(33)
+    for lens, Hq, Hkv in (([5, 17, 1, 33], 4, 2), ([40, 9], 6, 3), ([16], 2, 2)):
+        D, bs = 16, 4
+        k, v, ks, vs, bt, cl = _random_int8_paged(rng, lens, Hkv, D, bs)
+        q = rand_bits(rng, (len(lens), Hq, D))
+        got = orc.paged_attention_int8(q, k, v, ks, vs, bt, cl, 0.3)
+        kd = k.astype(np.float64) * ks.astype(np.float64)[..., None]
+        vd = v.astype(np.float64) * vs.astype(np.float64)[..., None]
+        G = Hq // Hkv
+        for b, L in enumerate(lens):
+            pages = bt[b, :-(-L // bs)]
+            K = np.transpose(kd[pages], (0, 2, 1, 3)).reshape(-1, Hkv, D)[:L]
+            V = np.transpose(vd[pages], (0, 2, 1, 3)).reshape(-1, Hkv, D)[:L]
+            K, V = np.repeat(K, G, axis=1), np.repeat(V, G, axis=1)
+            S = np.einsum("hd,jhd->hj", bf16_bits_to_f64(q[b]), K) * np.float64(np.float32(0.3))
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            ref = np.einsum("hj,jhd->hd", P / P.sum(axis=1, keepdims=True), V)
+            assert np.allclose(got[b], ref, rtol=1e-12, atol=1e-14), np.abs(got[b] - ref).max()
+
+
+def pin_int8_equals_bf16_path_on_exact_values(orc):
+    """Power-of-two scales make code * scale bf16-exact; the int8 decode then
+    equals the (pinned) bf16 decode of the same values bit for bit."""
+    rng = np.random.default_rng(34)
+    lens, Hq, Hkv, D, bs = [23, 7, 40], 8, 2, 32, 8
+    k, v, ks, vs, bt, cl = _random_int8_paged(rng, lens, Hkv, D, bs)
+    ks = np.ldexp(1.0, -rng.integers(4, 9, size=ks.shape)).astype(np.float32)
+    vs = np.ldexp(1.0, -rng.integers(4, 9, size=vs.shape)).astype(np.float32)
+    kb = f32_to_bf16_bits(k.astype(np.float32) * ks[..., None])
+    vb = f32_to_bf16_bits(v.astype(np.float32) * vs[..., None])
+    assert np.array_equal(bf16_bits_to_f64(kb), k.astype(np.float64) * ks[..., None])
+    q = rand_bits(rng, (len(lens), Hq, D))
+    a = orc.paged_attention_int8(q, k, v, ks, vs, bt, cl, 0.125)
+    b = orc.paged_attention(q, kb, vb, bt, cl, 0.125)
+    assert np.array_equal(a, b)
+
+
 ALL_PINS = [
     pin_golden_closed_form,
     pin_brute_force_decode,
@@ -336,4 +482,10 @@ ALL_PINS = [
     pin_gqa_equals_materialised_mha,
     pin_split_merge_equals_plain,
     pin_empty_context_is_zero,
+    pin_int8_exact_grid_rows,
+    pin_int8_ties_round_to_even,
+    pin_int8_error_within_half_step,
+    pin_int8_zero_row_and_slots,
+    pin_int8_attention_brute_force,
+    pin_int8_equals_bf16_path_on_exact_values,
 ]

@@ -4,14 +4,16 @@ The mutants are compile-time variants of the C oracle (PKV_ORACLE_MUTANT):
 1 interleaved GQA head map, 2 page/row index swapped, 3 scale dropped,
 4 causal edge off by one, 5 newest key dropped in decode, 6 softmax
 normaliser dropped, 7 token-major page layout, 8 cache-write slot off by one,
-9 scores taken against V, 10 merge weight sign flipped.
+9 scores taken against V, 10 merge weight sign flipped, 11 int8 code range
+128 instead of 127, 12 int8 rounding toward zero, 13 int8 V rows scaled by the
+K scale.
 """
 import pytest
 
 import oracle
 import oracle_pins
 
-MUTANTS = list(range(1, 11))
+MUTANTS = list(range(1, 14))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
