@@ -119,6 +119,46 @@ size_t pkv_paged_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv,
                                           int32_t max_context_len_hint);
 
 /*
+ * INT8 KV cache.  The Tiny-Infer page (section "推测性解码与INT8量化") names
+ * an INT8 KV cache as the way to halve its memory; it fixes neither the scale
+ * granularity nor the rounding.  This library's reading: symmetric codes with
+ * one fp32 scale per written row (one token's D values of one kv head), the
+ * granularity an incremental cache write can fix when the row is written:
+ *   amax = max |x|;  inv = 127 / amax;  code = clamp(rint(x * inv), -127, 127);
+ *   scale = amax / 127   (fp32, round half to even; amax = 0: codes 0, scale 0)
+ * and the row's value is code * scale.  Non-finite inputs give unspecified codes.
+ *   k_cache, v_cache : device, [NB][Hkv][bs][D] int8, 16-byte aligned
+ *   k_scale, v_scale : device, [NB][Hkv][bs] fp32, 16-byte aligned
+ * kv_cache_write_int8: key/value as for pkv_kv_cache_write (bf16, token
+ * strides in elements, 2-byte aligned); D in {64, 128, 256}; any bs.  Slots
+ * < 0 are skipped; a slot outside the pool sets PKV_ERR_BOUNDS on the device.
+ */
+pkv_status pkv_kv_cache_write_int8(const void* key, const void* value,
+                                   int64_t key_stride_tok,
+                                   int64_t value_stride_tok, void* k_cache,
+                                   void* v_cache, float* k_scale, float* v_scale,
+                                   const int64_t* slot_mapping, int32_t T,
+                                   int32_t Hkv, int32_t D, int32_t NB, int32_t bs,
+                                   pkv_stream_t stream);
+
+/*
+ * paged_attention_int8 -- pkv_paged_attention over the int8 cache: the same
+ * plan, launch shapes, workspace (pkv_paged_attention_workspace_size) and
+ * errors; K and V are read as codes and scaled by their row's scale inside
+ * the kernel (half the bytes of the bf16 cache, plus 4 bytes per row).
+ * q and out are bf16 as for pkv_paged_attention; D in {64, 128}, bs = 16.
+ */
+pkv_status pkv_paged_attention_int8(void* out, const void* q, const void* k_cache,
+                                    const void* v_cache, const float* k_scale,
+                                    const float* v_scale,
+                                    const int32_t* block_tables, int32_t MB,
+                                    const int32_t* context_lens, int32_t B,
+                                    int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                                    int32_t bs, float scale,
+                                    int32_t max_context_len_hint, void* workspace,
+                                    size_t workspace_bytes, pkv_stream_t stream);
+
+/*
  * paged_attention_split -- the split-KV ("flash-decoding") path with an
  * explicit split size.  Split c of sequence b covers logical pages
  * [c*pages_per_split, (c+1)*pages_per_split); each CTA writes its normalised

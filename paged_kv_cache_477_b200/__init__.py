@@ -13,6 +13,9 @@ Calls (same names as the C ABI):
     paged_attention_split(..., pages_per_split)
     paged_attention_prefill(q, query_start_loc, k_cache, v_cache, block_tables,
                             context_lens, scale, max_q_len, ...)
+    kv_cache_write_int8(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping)
+    paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                         context_lens, scale, ...)
 """
 from __future__ import annotations
 
@@ -48,6 +51,9 @@ EXPORTS = {
     "pkv_split_workspace_size": ([_I32, _I32, _I32, _I32], _SZ),
     "pkv_paged_attention_split_noalloc": ([_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                            _I32, _F32, _I32, _I32, _I32, _P], _I32),
+    "pkv_kv_cache_write_int8": ([_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
+    "pkv_paged_attention_int8": ([_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32,
+                                  _I32, _P, _SZ, _P], _I32),
     "pkv_paged_attention_prefill": ([_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                      _I32, _I32, _I32, _F32, _I32, _P], _I32),
     "pkv_get_device_error": ([_P, ctypes.POINTER(_I32)], _I32),
@@ -156,6 +162,65 @@ def _decode_common(q, k_cache, v_cache, block_tables, context_lens, out):
         if out.shape != q.shape:
             raise ValueError("out must have q's shape")
     return NB, Hkv, bs, D, B, Hq, block_tables.shape[1], out
+
+
+def kv_cache_write_int8(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping, stream=None) -> None:
+    """Quantise key/value [T, Hkv, D] (bf16, rows may be strided) into the int8
+    cache k_cache/v_cache [NB, Hkv, bs, D] and its fp32 row scales [NB, Hkv, bs]."""
+    for t, name in ((key, "key"), (value, "value")):
+        _dev(t, name, torch.bfloat16)
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be [T, Hkv, D] with contiguous (head, dim)")
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _contig(_dev(t, name, torch.int8), name)
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _contig(_dev(t, name, torch.float32), name)
+    _contig(_dev(slot_mapping, "slot_mapping", torch.int64), "slot_mapping")
+    T, Hkv, D = key.shape
+    NB, Hkv2, bs, D2 = k_cache.shape
+    if (Hkv2, D2) != (Hkv, D) or value.shape != key.shape or v_cache.shape != k_cache.shape \
+            or k_scale.shape != (NB, Hkv, bs) or v_scale.shape != k_scale.shape or slot_mapping.numel() != T:
+        raise ValueError("shape mismatch between key/value, caches, scales and slot_mapping")
+    rc = load_library().pkv_kv_cache_write_int8(
+        key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0), k_cache.data_ptr(),
+        v_cache.data_ptr(), k_scale.data_ptr(), v_scale.data_ptr(), slot_mapping.data_ptr(), T, Hkv, D, NB, bs,
+        _stream(stream))
+    _check(rc, "kv_cache_write_int8")
+
+
+def paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale: float,
+                         out=None, max_context_len: int = 0, workspace: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Decode over the int8 cache.  q [B, Hq, D] bf16 -> out [B, Hq, D] bf16."""
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _contig(_dev(t, name, torch.int8), name)
+    for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
+        _contig(_dev(t, name, torch.float32), name)
+    _contig(_dev(q, "q", torch.bfloat16), "q")
+    _contig(_dev(block_tables, "block_tables", torch.int32), "block_tables")
+    _contig(_dev(context_lens, "context_lens", torch.int32), "context_lens")
+    NB, Hkv, bs, D = k_cache.shape
+    B, Hq, Dq = q.shape
+    MB = block_tables.shape[1]
+    if Dq != D or v_cache.shape != k_cache.shape or k_scale.shape != (NB, Hkv, bs) or \
+            v_scale.shape != k_scale.shape or block_tables.shape[0] != B or context_lens.numel() != B:
+        raise ValueError("shape mismatch between q, caches, scales, block_tables and context_lens")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _contig(_dev(out, "out", torch.bfloat16), "out")
+    lib = load_library()
+    need = int(lib.pkv_paged_attention_workspace_size(B, Hq, Hkv, D, MB, bs, max_context_len))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.pkv_paged_attention_int8(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                      k_scale.data_ptr(), v_scale.data_ptr(), block_tables.data_ptr(), MB,
+                                      context_lens.data_ptr(), B, Hq, Hkv, D, NB, bs, float(scale),
+                                      int(max_context_len), ws_ptr, ws_bytes, _stream(stream))
+    _check(rc, "paged_attention_int8")
+    return out
 
 
 def workspace_size(B, Hq, Hkv, D, MB, bs=16, max_context_len: int = 0) -> int:

@@ -50,3 +50,80 @@ __global__ void __launch_bounds__(256) kv_cache_write_kernel(const __grid_consta
 }
 
 }  // namespace pkv
+
+namespace pkv {
+
+// ---------------------------------------------------------------------------
+// INT8 cache write: quantise each new (token, kv head) row of K and of V to
+// int8 codes with one fp32 scale per row (Tiny-Infer page, section on INT8
+// quantisation; the page fixes no granularity or rounding, so: symmetric,
+// amax / 127, round half to even, all in fp32 -- the same operations, in the
+// same order, as the reference definition, so codes and scales are exact).
+//   amax = max |x|;  inv = 127 / amax;  code = clamp(rint(x * inv), +-127);
+//   scale = amax / 127;  a zero row gives codes 0 and scale 0.
+// One warp per row (K rows, then V rows); lane l holds elements
+// [l * EPL, (l + 1) * EPL).  Non-finite inputs give unspecified codes.
+// ---------------------------------------------------------------------------
+struct KvWriteI8Params {
+  const __nv_bfloat16* key;    // [T][Hkv][D], token stride given
+  const __nv_bfloat16* value;
+  int64_t key_stride, value_stride;  // elements
+  int8_t* k_cache;             // [NB][Hkv][bs][D]
+  int8_t* v_cache;
+  float* k_scale;              // [NB][Hkv][bs]
+  float* v_scale;
+  const int64_t* slot_mapping;
+  int64_t rows;                // 2 * T * Hkv
+  int64_t pool_slots;          // NB * bs
+  int32_t T, Hkv, D, bs;
+};
+
+template <int EPL>
+__global__ void __launch_bounds__(256) kv_cache_write_i8_kernel(const __grid_constant__ KvWriteI8Params p) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.rows) return;
+  const bool is_v = row >= (int64_t)p.T * p.Hkv;
+  const int64_t th = is_v ? row - (int64_t)p.T * p.Hkv : row;
+  const int32_t h = (int32_t)(th % p.Hkv);
+  const int64_t t = th / p.Hkv;
+  const int64_t slot = __ldg(p.slot_mapping + t);
+  if (slot < 0) return;  // padding token
+  if (slot >= p.pool_slots) {
+    if (lane == 0) set_error(PKV_ERR_BOUNDS);
+    return;
+  }
+  const __nv_bfloat16* src = (is_v ? p.value + t * p.value_stride : p.key + t * p.key_stride) +
+                             (int64_t)h * p.D + lane * EPL;
+  float x[EPL];
+  float amax = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    x[e] = __bfloat162float(src[e]);
+    amax = fmaxf(amax, fabsf(x[e]));
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const int64_t blk = slot / p.bs, off = slot % p.bs;
+  const int64_t dst_row = (blk * p.Hkv + h) * p.bs + off;
+  int8_t* dst = (is_v ? p.v_cache : p.k_cache) + dst_row * p.D + lane * EPL;
+  const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+  int8_t c[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    const int r = __float2int_rn(__fmul_rn(x[e], inv));  // round half to even
+    c[e] = (int8_t)max(-127, min(127, r));
+  }
+  if constexpr (EPL == 2) {
+    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)((uint8_t)c[0] | ((uint8_t)c[1] << 8));
+  } else {
+#pragma unroll
+    for (int w = 0; w < EPL / 4; ++w)
+      reinterpret_cast<uint32_t*>(dst)[w] = (uint32_t)(uint8_t)c[4 * w] | ((uint32_t)(uint8_t)c[4 * w + 1] << 8) |
+                                            ((uint32_t)(uint8_t)c[4 * w + 2] << 16) |
+                                            ((uint32_t)(uint8_t)c[4 * w + 3] << 24);
+  }
+  if (lane == 0) (is_v ? p.v_scale : p.k_scale)[dst_row] = amax > 0.f ? __fdiv_rn(amax, 127.f) : 0.f;
+}
+
+}  // namespace pkv

@@ -50,18 +50,21 @@ size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // ----------------------------------------------------------------- decode --
 constexpr int kDecodeWarps = 4;
-// pages per ring stage: two for D=64, so a stage is 32 key rows and a lane
-// works on four rows per step whatever D is
-constexpr int pages_per_stage(int D) { return D == 128 ? 1 : 2; }
-// stages per warp: 3 x 8 KB -> 96 KB of pages in flight per CTA, two CTAs per SM
-constexpr int stages_for(int D) { return 3; }
+// pages per ring stage: one 8 KB bf16 page pair at D=128, otherwise two, so a
+// stage is 32 key rows whenever a page is smaller and a lane always works on
+// four rows per step
+constexpr int pages_per_stage(int D, bool I8) { return (D == 128 && !I8) ? 1 : 2; }
+// stages per warp: ~96-104 KB of pages in flight per CTA, two CTAs per SM
+// (3 x 8 KB bf16, 3 x 8.25 KB int8 at D=128, 6 x 4.25 KB int8 at D=64)
+constexpr int stages_for(int D, bool I8) { return (I8 && D == 64) ? 6 : 3; }
 
-template <int D, int HG>
-using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D), pages_per_stage(D)>;
+template <int D, int HG, bool I8 = false>
+using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D, I8), pages_per_stage(D, I8), I8>;
 
-template <int D, int HG>
+template <int D, int HG, bool I8 = false>
 struct DecodeKernel {
-  static constexpr auto fn = pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D), pages_per_stage(D)>;
+  static constexpr auto fn =
+      pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D, I8), pages_per_stage(D, I8), I8>;
   // set the dynamic shared-memory limit once per device; return CTAs per SM
   static int prepare(int dev) {
     static int occ[kMaxDevices] = {0};
@@ -70,13 +73,13 @@ struct DecodeKernel {
     std::lock_guard<std::mutex> g(mu);
     if (occ[dev] == 0) {
       if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess ||
+                               DecodeS<D, HG, I8>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return -1;
       int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DecodeS<D, HG>::THREADS,
-                                                        DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess ||
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DecodeS<D, HG, I8>::THREADS,
+                                                        DecodeS<D, HG, I8>::SMEM_BYTES) != cudaSuccess ||
           n <= 0)
         return -1;
       occ[dev] = n;
@@ -151,13 +154,25 @@ DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, 
   return pl;
 }
 
-template <int D, int HG>
+template <int D, int HG, bool I8 = false>
 pkv_status launch_decode_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C,
                            cudaStream_t st) {
-  if (DecodeKernel<D, HG>::prepare(current_device()) < 0) return PKV_ERR_CUDA;
+  if (DecodeKernel<D, HG, I8>::prepare(current_device()) < 0) return PKV_ERR_CUDA;
   dim3 grid(C, Hkv * nsub, B);
-  DecodeKernel<D, HG>::fn<<<grid, DecodeS<D, HG>::THREADS, DecodeS<D, HG>::SMEM_BYTES, st>>>(p);
+  DecodeKernel<D, HG, I8>::fn<<<grid, DecodeS<D, HG, I8>::THREADS, DecodeS<D, HG, I8>::SMEM_BYTES, st>>>(p);
   return launch_status();
+}
+
+template <bool I8>
+pkv_status launch_decode_any(const pkv::DecodeParams& p, int D, int HG, int B, int Hkv, int nsub, int C,
+                             cudaStream_t st) {
+  if (D == 128)
+    return HG == 4 ? launch_decode_t<128, 4, I8>(p, B, Hkv, nsub, C, st)
+           : HG == 2 ? launch_decode_t<128, 2, I8>(p, B, Hkv, nsub, C, st)
+                     : launch_decode_t<128, 1, I8>(p, B, Hkv, nsub, C, st);
+  return HG == 4 ? launch_decode_t<64, 4, I8>(p, B, Hkv, nsub, C, st)
+         : HG == 2 ? launch_decode_t<64, 2, I8>(p, B, Hkv, nsub, C, st)
+                   : launch_decode_t<64, 1, I8>(p, B, Hkv, nsub, C, st);
 }
 
 template <int D>
@@ -183,10 +198,12 @@ pkv_status check_decode_args(void* out, const void* q, const void* k_cache, cons
   return PKV_OK;
 }
 
+// k_scale / v_scale non-null: the int8 cache (codes in k_cache / v_cache).
 pkv_status run_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
                       const int32_t* block_tables, int32_t MB, const int32_t* context_lens,
                       int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB, float scale,
-                      const DecodePlan& pl, void* workspace, cudaStream_t st) {
+                      const DecodePlan& pl, void* workspace, cudaStream_t st,
+                      const float* k_scale = nullptr, const float* v_scale = nullptr) {
   const int G = Hq / Hkv, HG = heads_per_cta(G), nsub = G / HG;
   const int C = pl.num_splits;
   pkv::DecodeParams p{};
@@ -194,6 +211,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.k_cache = static_cast<const unsigned char*>(k_cache);
   p.v_cache = static_cast<const unsigned char*>(v_cache);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NB = NB; p.MB = MB;
@@ -208,15 +227,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
     p.lse_part = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) +
                                           round256(rows * D * sizeof(float)));
   }
-  pkv_status s;
-  if (D == 128)
-    s = HG == 4 ? launch_decode_t<128, 4>(p, B, Hkv, nsub, C, st)
-        : HG == 2 ? launch_decode_t<128, 2>(p, B, Hkv, nsub, C, st)
-                  : launch_decode_t<128, 1>(p, B, Hkv, nsub, C, st);
-  else
-    s = HG == 4 ? launch_decode_t<64, 4>(p, B, Hkv, nsub, C, st)
-        : HG == 2 ? launch_decode_t<64, 2>(p, B, Hkv, nsub, C, st)
-                  : launch_decode_t<64, 1>(p, B, Hkv, nsub, C, st);
+  pkv_status s = k_scale ? launch_decode_any<true>(p, D, HG, B, Hkv, nsub, C, st)
+                         : launch_decode_any<false>(p, D, HG, B, Hkv, nsub, C, st);
   if (s != PKV_OK) return s;
   int launches = 1;
   if (C > 1) {
@@ -353,6 +365,70 @@ pkv_status pkv_kv_cache_write(const void* key, const void* value, int64_t key_st
   pkv_status s = launch_status();
   if (s == PKV_OK) t_launches = 1;
   return s;
+}
+
+pkv_status pkv_kv_cache_write_int8(const void* key, const void* value, int64_t key_stride_tok,
+                                   int64_t value_stride_tok, void* k_cache, void* v_cache, float* k_scale,
+                                   float* v_scale, const int64_t* slot_mapping, int32_t T, int32_t Hkv,
+                                   int32_t D, int32_t NB, int32_t bs, pkv_stream_t stream) {
+  t_launches = 0;
+  if (T < 0 || Hkv <= 0 || D <= 0 || NB < 0 || bs <= 0) return PKV_ERR_INVALID_ARG;
+  if (D != 64 && D != 128 && D != 256) return PKV_ERR_UNSUPPORTED;
+  if (T == 0) return PKV_OK;
+  if (!key || !value || !k_cache || !v_cache || !k_scale || !v_scale || !slot_mapping)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_scale) || !aligned16(v_scale) ||
+      (reinterpret_cast<uintptr_t>(key) & 1) || (reinterpret_cast<uintptr_t>(value) & 1))
+    return PKV_ERR_INVALID_ARG;
+  if (key_stride_tok < (int64_t)Hkv * D || value_stride_tok < (int64_t)Hkv * D) return PKV_ERR_INVALID_ARG;
+  pkv::KvWriteI8Params p{};
+  p.key = static_cast<const __nv_bfloat16*>(key);
+  p.value = static_cast<const __nv_bfloat16*>(value);
+  p.key_stride = key_stride_tok;
+  p.value_stride = value_stride_tok;
+  p.k_cache = static_cast<int8_t*>(k_cache);
+  p.v_cache = static_cast<int8_t*>(v_cache);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.slot_mapping = slot_mapping;
+  p.rows = 2 * (int64_t)T * Hkv;
+  p.pool_slots = (int64_t)NB * bs;
+  p.T = T; p.Hkv = Hkv; p.D = D; p.bs = bs;
+  const int64_t blocks = (p.rows + 7) / 8;  // one warp per row, 8 warps per block
+  if (blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64)
+    pkv::kv_cache_write_i8_kernel<2><<<(unsigned)blocks, 256, 0, st>>>(p);
+  else if (D == 128)
+    pkv::kv_cache_write_i8_kernel<4><<<(unsigned)blocks, 256, 0, st>>>(p);
+  else
+    pkv::kv_cache_write_i8_kernel<8><<<(unsigned)blocks, 256, 0, st>>>(p);
+  pkv_status s = launch_status();
+  if (s == PKV_OK) t_launches = 1;
+  return s;
+}
+
+pkv_status pkv_paged_attention_int8(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                    const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                    int32_t MB, const int32_t* context_lens, int32_t B, int32_t Hq,
+                                    int32_t Hkv, int32_t D, int32_t NB, int32_t bs, float scale,
+                                    int32_t max_context_len_hint, void* workspace, size_t workspace_bytes,
+                                    pkv_stream_t stream) {
+  t_launches = 0;
+  pkv_status s = check_decode_args(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq,
+                                    Hkv, D, NB, bs, PKV_BF16);
+  if (s != PKV_OK || B == 0) return s;
+  if (MB > 0 && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale)))
+    return PKV_ERR_INVALID_ARG;
+  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint);
+  if (pl.num_splits > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned16(workspace)))
+    pl = DecodePlan{1, std::max<int32_t>(MB, 1), 0};  // no room: one CTA per head group
+  if (pl.num_splits == 1) pl.pages_per_split = std::max<int32_t>(MB, 1);
+  // a never-read dummy keeps the kernel on its int8 path when MB = 0
+  static const float kNoScale[4] = {0.f, 0.f, 0.f, 0.f};
+  return run_decode(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq, Hkv, D, NB, scale, pl,
+                    workspace, static_cast<cudaStream_t>(stream), k_scale ? k_scale : kNoScale,
+                    v_scale ? v_scale : kNoScale);
 }
 
 size_t pkv_split_workspace_size(int32_t B, int32_t Hq, int32_t D, int32_t num_splits) {

@@ -18,6 +18,11 @@ Recipe (one case):
    tail of each sequence's last page, and the slots the write step is about to
    fill -- holds bf16 NaN, so an over-read or a missed write shows up as NaN.
 5. ``scale = 1 / sqrt(D)`` computed in float32.
+6. ``kv_dtype="int8"``: the pool holds int8 codes drawn uniformly from
+   [-127, 127] and one fp32 scale per row drawn log-uniformly from
+   [0.008, 0.03] (so values code * scale are of order 1); canary rows get a
+   NaN scale.  No quantisation happens here: the new rows of the write step
+   are bf16 N(0, 1) as above, and the write step quantises them.
 
 The five named workloads reproduce the attention shapes of the pages' models
 (Llama-3.2-1B and Llama-3-8B) as stand-ins: the pages measure on no dataset.
@@ -58,13 +63,19 @@ class PagedCase:
     query_start_loc: Optional[torch.Tensor] = None  # prefill [B+1] int32
     max_q_len: int = 1
     lens: list = field(default_factory=list)
+    kv_dtype: str = "bf16"         # "int8": k_cache/v_cache hold int8 codes
+    k_scale: Optional[torch.Tensor] = None    # int8: [NB, Hkv, bs] fp32 row scales
+    v_scale: Optional[torch.Tensor] = None
 
     @property
     def G(self) -> int:
         return self.Hq // self.Hkv
 
     def kv_bytes_read(self) -> int:
-        """K and V bytes a decode pass must read: sum_b L_b * Hkv * D * 2 B * 2."""
+        """K and V bytes a decode pass must read: sum_b L_b * Hkv * D * 2 B * 2
+        (int8: sum_b L_b * Hkv * (D + 4) * 2, codes plus the row scale)."""
+        if self.kv_dtype == "int8":
+            return int(sum(self.lens)) * self.Hkv * (self.D + 4) * 2
         return int(sum(self.lens)) * self.Hkv * self.D * 2 * 2
 
 
@@ -76,7 +87,7 @@ def make_case(*, name: str = "custom", kind: str = "decode", B: int, Hq: int, Hk
               D: int, bs: int = 16, lens: Sequence[int], seed: int, device="cpu",
               pool_blocks: Optional[int] = None, MB: Optional[int] = None,
               write_tokens: int = 0, q_len: Optional[Sequence[int]] = None,
-              canaries: bool = True, scale: Optional[float] = None) -> PagedCase:
+              canaries: bool = True, scale: Optional[float] = None, kv_dtype: str = "bf16") -> PagedCase:
     """Build one seeded case.
 
     kind="decode": one query per sequence; the last ``write_tokens`` positions
@@ -126,8 +137,18 @@ def make_case(*, name: str = "custom", kind: str = "decode", B: int, Hq: int, Hk
         return out
 
     q = randn_bf16(nq, Hq, D)
-    k_cache = randn_bf16(NB, Hkv, bs, D)
-    v_cache = randn_bf16(NB, Hkv, bs, D)
+    k_scale = v_scale = None
+    if kv_dtype == "int8":
+        assert kind == "decode", "the int8 cache is read by decode only"
+        k_cache = torch.randint(-127, 128, (NB, Hkv, bs, D), generator=gd, device=device, dtype=torch.int8)
+        v_cache = torch.randint(-127, 128, (NB, Hkv, bs, D), generator=gd, device=device, dtype=torch.int8)
+        lo, hi = math.log(0.008), math.log(0.03)
+        k_scale = torch.exp(lo + (hi - lo) * torch.rand(NB, Hkv, bs, generator=gd, device=device))
+        v_scale = torch.exp(lo + (hi - lo) * torch.rand(NB, Hkv, bs, generator=gd, device=device))
+    else:
+        assert kv_dtype == "bf16"
+        k_cache = randn_bf16(NB, Hkv, bs, D)
+        v_cache = randn_bf16(NB, Hkv, bs, D)
     T = sum(len(w) for w in write_pos)
     new_key = new_value = slot_mapping = None
     if T > 0:
@@ -148,10 +169,15 @@ def make_case(*, name: str = "custom", kind: str = "decode", B: int, Hq: int, Hk
                 if hi > lo:
                     valid[int(bt[b, p]), : hi - lo] = True
         invalid = (~valid).to(device)                          # [NB, bs]
-        nanv = torch.tensor(float("nan"), dtype=torch.bfloat16, device=device)
-        mask = invalid[:, None, :, None]
-        k_cache = torch.where(mask, nanv, k_cache)
-        v_cache = torch.where(mask, nanv, v_cache)
+        if kv_dtype == "int8":
+            nanf = torch.tensor(float("nan"), dtype=torch.float32, device=device)
+            k_scale = torch.where(invalid[:, None, :], nanf, k_scale)
+            v_scale = torch.where(invalid[:, None, :], nanf, v_scale)
+        else:
+            nanv = torch.tensor(float("nan"), dtype=torch.bfloat16, device=device)
+            mask = invalid[:, None, :, None]
+            k_cache = torch.where(mask, nanv, k_cache)
+            v_cache = torch.where(mask, nanv, v_cache)
 
     qsl = None
     if kind == "prefill":
@@ -165,7 +191,9 @@ def make_case(*, name: str = "custom", kind: str = "decode", B: int, Hq: int, Hk
         new_key=new_key, new_value=new_value,
         slot_mapping=slot_mapping.to(device) if slot_mapping is not None else None,
         query_start_loc=qsl.to(device) if qsl is not None else None,
-        max_q_len=max(qlens) if qlens else 0, lens=lens,
+        max_q_len=max(qlens) if qlens else 0, lens=lens, kv_dtype=kv_dtype,
+        k_scale=k_scale.contiguous() if k_scale is not None else None,
+        v_scale=v_scale.contiguous() if v_scale is not None else None,
     )
 
 
@@ -200,6 +228,11 @@ WORKLOADS = {
         write_tokens=1,
         desc="Llama-3-8B-shaped decode: B=128, Hq=32/Hkv=8, D=128, bs=16, ctx 4096, "
              "one new token written per sequence before attention"),
+    "llama3_8b_decode_int8": dict(
+        kind="decode", B=128, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 128, seed=1006,
+        write_tokens=1, kv_dtype="int8",
+        desc="Llama-3-8B-shaped decode over an INT8 cache (one fp32 scale per row): B=128, Hq=32/Hkv=8, "
+             "D=128, bs=16, ctx 4096, one new token quantised into the cache per sequence before attention"),
     "ragged_long_decode": dict(
         kind="decode", B=16, Hq=32, Hkv=8, D=128, bs=16, lens=_lens_ragged(1004), seed=1004,
         desc="ragged long-context decode: B=16, Hq=32/Hkv=8, D=128, 4 x 32768 + 12 log-uniform "

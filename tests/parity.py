@@ -38,8 +38,15 @@ class HostCase:
     def __init__(self, case: PagedCase):
         self.case = case
         self.q = bf16_bits(case.q)
-        self.k = bf16_bits(case.k_cache).copy()
-        self.v = bf16_bits(case.v_cache).copy()
+        self.int8 = case.kv_dtype == "int8"
+        if self.int8:
+            self.k = case.k_cache.cpu().numpy().copy()
+            self.v = case.v_cache.cpu().numpy().copy()
+            self.ks = case.k_scale.cpu().numpy().copy()
+            self.vs = case.v_scale.cpu().numpy().copy()
+        else:
+            self.k = bf16_bits(case.k_cache).copy()
+            self.v = bf16_bits(case.v_cache).copy()
         self.bt = case.block_tables.cpu().numpy().astype(np.int32)
         self.lens = case.context_lens.cpu().numpy().astype(np.int32)
         self.qsl = case.query_start_loc.cpu().numpy().astype(np.int32) if case.query_start_loc is not None else None
@@ -48,13 +55,21 @@ class HostCase:
     def apply_write(self):
         c = self.case
         if c.new_key is not None and not self.written:
-            oracle.get().kv_cache_write(bf16_bits(c.new_key), bf16_bits(c.new_value), self.k, self.v,
-                                        c.slot_mapping.cpu().numpy().astype(np.int64))
+            slots = c.slot_mapping.cpu().numpy().astype(np.int64)
+            if self.int8:
+                oracle.get().kv_cache_write_int8(bf16_bits(c.new_key), bf16_bits(c.new_value), self.k, self.v,
+                                                 self.ks, self.vs, slots)
+            else:
+                oracle.get().kv_cache_write(bf16_bits(c.new_key), bf16_bits(c.new_value), self.k, self.v, slots)
         self.written = True
         return self
 
     def decode_ref(self, rows=None):
         rows = np.arange(self.case.B) if rows is None else np.asarray(rows)
+        if self.int8:
+            return oracle.get().paged_attention_int8(np.ascontiguousarray(self.q[rows]), self.k, self.v, self.ks,
+                                                     self.vs, np.ascontiguousarray(self.bt[rows]),
+                                                     np.ascontiguousarray(self.lens[rows]), self.case.scale)
         return oracle.get().paged_attention(np.ascontiguousarray(self.q[rows]), self.k, self.v,
                                             np.ascontiguousarray(self.bt[rows]),
                                             np.ascontiguousarray(self.lens[rows]), self.case.scale)
