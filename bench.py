@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--profile", default=None,
-                    choices=["decode", "decode_full", "decode_d64", "split", "prefill", "write"],
+                    choices=["decode", "decode_full", "decode_d64", "decode_int8", "split", "prefill", "write"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
@@ -323,6 +323,23 @@ def extras(peaks):
                      "l2": "inputs larger than L2"}
         del c, out, ws
         torch.cuda.empty_cache()
+    # INT8 cache (one fp32 scale per row): same shape as the headline step
+    c = wl.workload("llama3_8b_decode_int8", device="cuda")
+    pkv.kv_cache_write_int8(c.new_key, c.new_value, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.slot_mapping)
+    out = torch.empty_like(c.q)
+    ws = torch.empty(max(1, pkv.workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, 4096)), dtype=torch.uint8,
+                     device="cuda")
+    fn = lambda: pkv.paged_attention_int8(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_tables,
+                                          c.context_lens, c.scale, out=out, max_context_len=4096, workspace=ws)
+    time_calls(fn, 3)
+    ms = statistics.median(time_calls(fn, 20))
+    gbs = decode_bytes(c) / (ms * 1e-3) / 1e9
+    res["llama3_8b_decode_int8"] = {"GB/s": round(gbs, 1), "us": round(ms * 1e3, 2),
+                                    "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "launches": pkv.last_launch_count(),
+                                    "bytes": decode_bytes(c), "kv_bytes_vs_bf16": 0.5 + 2.0 / c.D,
+                                    "l2": "inputs larger than L2"}
+    del c, out, ws
+    torch.cuda.empty_cache()
     c = wl.workload("chunked_prefill", device="cuda")
     pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)
     out = torch.empty_like(c.q)
@@ -367,6 +384,14 @@ def profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
                                 max_context_len=4096)
+    elif kind == "decode_int8":
+        # 32 of the Llama-3-8B-shaped sequences over the INT8 cache: 264 MiB of codes and scales
+        c = wl.make_case(B=32, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 32, seed=1006, device="cuda",
+                         kv_dtype="int8")
+        out = torch.empty_like(c.q)
+        for _ in range(launches):
+            pkv.paged_attention_int8(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_tables,
+                                     c.context_lens, c.scale, out=out, max_context_len=4096)
     elif kind in ("decode", "split", "write"):
         # 32 of the Llama-3-8B-shaped sequences: 512 MiB of K/V
         c = wl.make_case(B=32, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 32, seed=1003, device="cuda",
