@@ -84,9 +84,14 @@ class Oracle:
                                                 _I32, _I32]
         lib.ref_paged_attention_int8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32,
                                                  _I32, _I32, _F32]
+        lib.ref_paged_attention_window.argtypes = [_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
+                                                   _I32, _F32, _I32]
+        lib.ref_paged_attention_prefill_window.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
+                                                           _I32, _I32, _I32, _F32, _I32]
         for f in ("ref_kv_cache_write", "ref_paged_attention", "ref_contiguous_attention",
                   "ref_paged_attention_prefill", "ref_decode_partials", "ref_lse_merge",
-                  "ref_kv_cache_write_int8", "ref_paged_attention_int8"):
+                  "ref_kv_cache_write_int8", "ref_paged_attention_int8", "ref_paged_attention_window",
+                  "ref_paged_attention_prefill_window"):
             getattr(lib, f).restype = ctypes.c_int
         self.lib = lib
         self.mutant = lib.ref_mutant_id()
@@ -144,6 +149,39 @@ class Oracle:
                                                _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
                                                MB, _ptr(context_lens), B, Hq, Hkv, D, NB, bs, float(scale))
         self._check(rc, "paged_attention_int8", allow_bounds)
+        return out
+
+    # -- sliding window -------------------------------------------------------
+    def paged_attention_window(self, q, k_cache, v_cache, block_tables, context_lens, scale, window,
+                               allow_bounds=False) -> np.ndarray:
+        """Decode where the query (position L_b - 1) sees only its last ``window`` keys."""
+        B, Hq, D = q.shape
+        NB, Hkv, bs, _ = k_cache.shape
+        block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+        context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+        MB = block_tables.shape[1] if block_tables.ndim == 2 else 0
+        out = np.zeros((B, Hq, D), dtype=np.float64)
+        rc = self.lib.ref_paged_attention_window(_ptr(out), _ptr(np.ascontiguousarray(q)), _ptr(k_cache),
+                                                 _ptr(v_cache), _ptr(block_tables), MB, _ptr(context_lens),
+                                                 B, Hq, Hkv, D, NB, bs, float(scale), int(window))
+        self._check(rc, "paged_attention_window", allow_bounds)
+        return out
+
+    def paged_attention_prefill_window(self, q, query_start_loc, k_cache, v_cache, block_tables, context_lens,
+                                       scale, window, allow_bounds=False) -> np.ndarray:
+        sumQ, Hq, D = q.shape
+        NB, Hkv, bs, _ = k_cache.shape
+        B = len(context_lens)
+        block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+        qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+        context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+        MB = block_tables.shape[1] if block_tables.ndim == 2 else 0
+        out = np.zeros((sumQ, Hq, D), dtype=np.float64)
+        rc = self.lib.ref_paged_attention_prefill_window(_ptr(out), _ptr(np.ascontiguousarray(q)), _ptr(qsl),
+                                                         _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), MB,
+                                                         _ptr(context_lens), B, Hq, Hkv, D, NB, bs, float(scale),
+                                                         int(window))
+        self._check(rc, "paged_attention_prefill_window", allow_bounds)
         return out
 
     # -- decode ----------------------------------------------------------------

@@ -591,3 +591,126 @@ int ref_paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cac
   }
   return status;
 }
+
+/* ========================================================================= */
+/* Sliding-window attention over the paged cache.                             */
+/*                                                                            */
+/* A sliding-window cache is one of the KV cache variants the inference-lab  */
+/* page lists, an approximation for tight memory ("从零开始的LLM推理优化实验  */
+/* 室：从PyTorch基线到Triton内核的完整实践", section "KV缓存实验与长上下文   */
+/* 优化").  It gives no semantics; reading taken: a query at absolute         */
+/* position p sees the W keys p - W < j <= p (all of them if fewer exist).    */
+/* The result is plain attention over that key range, so the oracle gathers  */
+/* exactly those keys.                                                        */
+/* ========================================================================= */
+
+/* first key a query at absolute position p sees under window W (W >= 1) */
+static int64_t window_start(int64_t p, int32_t W) {
+#if PKV_ORACLE_MUTANT == 14
+  const int64_t j0 = p - W; /* planted: one key too many */
+#else
+  const int64_t j0 = p - W + 1;
+#endif
+  return j0 > 0 ? j0 : 0;
+}
+
+/* Decode: the query sits at position L_b - 1; out [B][Hq][D]. */
+int ref_paged_attention_window(double* out, const uint16_t* q, const uint16_t* k_cache,
+                               const uint16_t* v_cache, const int32_t* block_tables,
+                               int32_t MB, const int32_t* context_lens, int32_t B,
+                               int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                               int32_t bs, float scale, int32_t window) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || MB < 0 ||
+      Hq % Hkv != 0 || window < 1)
+    return ORC_INVALID;
+  for (int32_t b = 0; b < B; ++b)
+    if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)MB * bs)
+      return ORC_INVALID;
+  int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < (int64_t)B * Hq; ++bh) {
+    const int32_t b = (int32_t)(bh / Hq), h = (int32_t)(bh % Hq);
+    const int64_t L = context_lens[b];
+    const int64_t j0 = L > 0 ? window_start(L - 1, window) : 0;
+    const int64_t n = L - j0;
+    const int32_t g = kv_head_of(h, Hq, Hkv);
+    const uint16_t** kr = (const uint16_t**)malloc(sizeof(void*) * (n + 1));
+    const uint16_t** vr = (const uint16_t**)malloc(sizeof(void*) * (n + 1));
+    double* s = (double*)malloc(sizeof(double) * (n + 1));
+    double* qd = (double*)malloc(sizeof(double) * D);
+    int bad = 0;
+    for (int64_t j = 0; j < n; ++j) {
+      kr[j] = paged_row(k_cache, block_tables, MB, b, j0 + j, g, Hkv, D, NB, bs);
+      vr[j] = paged_row(v_cache, block_tables, MB, b, j0 + j, g, Hkv, D, NB, bs);
+      if (!kr[j] || !vr[j]) bad = 1;
+    }
+    double* o = out + bh * D;
+    if (bad) {
+      for (int32_t d = 0; d < D; ++d) o[d] = NAN;
+#pragma omp atomic write
+      status = ORC_BOUNDS;
+    } else {
+      widen_row(qd, q + bh * D, D);
+      attend_row(o, qd, D, (double)scale, kr, vr, n, s);
+    }
+    free(kr); free(vr); free(s); free(qd);
+  }
+  return status;
+}
+
+/* Chunked prefill: query i of sequence b sits at p = L_b - Q_b + i and sees
+ * keys window_start(p, W) .. p. */
+int ref_paged_attention_prefill_window(double* out, const uint16_t* q,
+                                       const int32_t* query_start_loc,
+                                       const uint16_t* k_cache, const uint16_t* v_cache,
+                                       const int32_t* block_tables, int32_t MB,
+                                       const int32_t* context_lens, int32_t B,
+                                       int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                                       int32_t bs, float scale, int32_t window) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || MB < 0 ||
+      Hq % Hkv != 0 || window < 1)
+    return ORC_INVALID;
+  if (query_start_loc[0] != 0) return ORC_INVALID;
+  for (int32_t b = 0; b < B; ++b) {
+    const int32_t Qb = query_start_loc[b + 1] - query_start_loc[b];
+    if (Qb < 0 || context_lens[b] < Qb ||
+        (int64_t)context_lens[b] > (int64_t)MB * bs)
+      return ORC_INVALID;
+  }
+  const int64_t sumQ = query_start_loc[B];
+  int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t th = 0; th < sumQ * Hq; ++th) {
+    const int64_t t = th / Hq;
+    const int32_t h = (int32_t)(th % Hq);
+    int32_t b = 0;
+    while (query_start_loc[b + 1] <= t) ++b;
+    const int64_t i = t - query_start_loc[b];
+    const int64_t Qb = query_start_loc[b + 1] - query_start_loc[b];
+    const int64_t p = context_lens[b] - Qb + i;
+    const int64_t j0 = window_start(p, window);
+    const int64_t n = p + 1 - j0;
+    const int32_t g = kv_head_of(h, Hq, Hkv);
+    const uint16_t** kr = (const uint16_t**)malloc(sizeof(void*) * (n + 1));
+    const uint16_t** vr = (const uint16_t**)malloc(sizeof(void*) * (n + 1));
+    double* s = (double*)malloc(sizeof(double) * (n + 1));
+    double* qd = (double*)malloc(sizeof(double) * D);
+    int bad = 0;
+    for (int64_t j = 0; j < n; ++j) {
+      kr[j] = paged_row(k_cache, block_tables, MB, b, j0 + j, g, Hkv, D, NB, bs);
+      vr[j] = paged_row(v_cache, block_tables, MB, b, j0 + j, g, Hkv, D, NB, bs);
+      if (!kr[j] || !vr[j]) bad = 1;
+    }
+    double* o = out + th * D;
+    if (bad) {
+      for (int32_t d = 0; d < D; ++d) o[d] = NAN;
+#pragma omp atomic write
+      status = ORC_BOUNDS;
+    } else {
+      widen_row(qd, q + th * D, D);
+      attend_row(o, qd, D, (double)scale, kr, vr, n, s);
+    }
+    free(kr); free(vr); free(s); free(qd);
+  }
+  return status;
+}

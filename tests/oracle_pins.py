@@ -28,7 +28,12 @@ section "分页KV缓存：借鉴操作系统的内存管理"; exact softmax atte
   exactly k and 2^-e; ties round to even; every value is within scale/2 of
   its code; a zero row gives zero codes and scale; attention over the int8
   pool equals NumPy brute force over the dequantised values, and equals the
-  pinned bf16 path bit for bit when the values are bf16-exact.
+  pinned bf16 path bit for bit when the values are bf16-exact;
+* sliding window W (a query at p sees keys p - W < j <= p; the reading of the
+  inference-lab page's sliding-window cache): W >= L is full attention bit for
+  bit, W = 1 returns the last key's V row, decode equals full attention over a
+  contiguous cache holding only the last W keys, the last query of a prefill
+  chunk equals windowed decode, and NumPy brute force with a banded mask agrees.
 """
 from __future__ import annotations
 
@@ -468,6 +473,77 @@ def pin_int8_equals_bf16_path_on_exact_values(orc):
     assert np.array_equal(a, b)
 
 
+# --------------------------------------------------------------------------- #
+# sliding window                                                               #
+# --------------------------------------------------------------------------- #
+
+def pin_window_covering_all_is_full_attention(orc):
+    rng = np.random.default_rng(41)
+    lens = [1, 9, 30, 17]
+    k, v, bt, cl = make_paged(rng, lens, 2, 16, 4)
+    q = rand_bits(rng, (4, 4, 16))
+    full = orc.paged_attention(q, k, v, bt, cl, 0.4)
+    for W in (30, 31, 1000):
+        assert np.array_equal(orc.paged_attention_window(q, k, v, bt, cl, 0.4, W), full)
+
+
+def pin_window_one_returns_last_v(orc):
+    rng = np.random.default_rng(42)
+    lens = [5, 12, 33]
+    k, v, bt, cl = make_paged(rng, lens, 1, 8, 4)
+    q = rand_bits(rng, (3, 2, 8))
+    out = orc.paged_attention_window(q, k, v, bt, cl, 0.7, 1)
+    for b, L in enumerate(lens):
+        blk = bt[b, (L - 1) // 4]
+        last_v = bf16_bits_to_f64(v[blk, 0, (L - 1) % 4])
+        assert np.array_equal(out[b, 0], last_v) and np.array_equal(out[b, 1], last_v)
+
+
+def pin_window_equals_truncated_context(orc):
+    """Windowed decode over L keys == full decode of a contiguous cache that
+    holds only the last W of them (same rows, same order: bit for bit)."""
+    rng = np.random.default_rng(43)
+    lens, Hq, Hkv, D, bs, W = [50, 7, 33, 16], 6, 3, 16, 4, 13
+    k, v, bt, cl = make_paged(rng, lens, Hkv, D, bs)
+    q = rand_bits(rng, (len(lens), Hq, D))
+    got = orc.paged_attention_window(q, k, v, bt, cl, 0.3, W)
+    n = [min(L, W) for L in lens]
+    kc = np.zeros((len(lens), max(n), Hkv, D), np.uint16)
+    vc = np.zeros_like(kc)
+    for b, L in enumerate(lens):
+        for i, j in enumerate(range(L - n[b], L)):
+            blk, row = bt[b, j // bs], j % bs
+            kc[b, i] = k[blk, :, row]
+            vc[b, i] = v[blk, :, row]
+    ref = orc.contiguous_attention(q, kc, vc, np.array(n, np.int32), 0.3)
+    assert np.array_equal(got, ref)
+
+
+def pin_window_prefill_brute_force_and_last_row(orc):
+    rng = np.random.default_rng(44)
+    lens, qlens, Hq, Hkv, D, bs = [40, 9, 25], [12, 9, 1], 4, 2, 16, 4
+    k, v, bt, cl = make_paged(rng, lens, Hkv, D, bs)
+    qsl = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = rand_bits(rng, (int(qsl[-1]), Hq, D))
+    for W in (1, 5, 16, 100):
+        got = orc.paged_attention_prefill_window(q, qsl, k, v, bt, cl, 0.25, W)
+        for b, (L, Q) in enumerate(zip(lens, qlens)):
+            K = brute.dense_kv(k, bt[b], L)
+            V = brute.dense_kv(v, bt[b], L)
+            G = Hq // Hkv
+            K, V = np.repeat(K, G, axis=1), np.repeat(V, G, axis=1)
+            qb = bf16_bits_to_f64(q[qsl[b]:qsl[b + 1]])
+            S = np.einsum("ihd,jhd->hij", qb, K) * np.float64(np.float32(0.25))
+            pos = L - Q + np.arange(Q)[:, None]
+            j = np.arange(L)[None, :]
+            S = np.where((j <= pos) & (j > pos - W), S, -np.inf)
+            P = np.exp(S - S.max(axis=-1, keepdims=True))
+            ref = np.einsum("hij,jhd->ihd", P / P.sum(axis=-1, keepdims=True), V)
+            assert np.allclose(got[qsl[b]:qsl[b + 1]], ref, rtol=1e-12, atol=1e-14)
+            last = orc.paged_attention_window(q[qsl[b + 1] - 1][None], k, v, bt[b:b + 1], cl[b:b + 1], 0.25, W)
+            assert np.array_equal(got[qsl[b + 1] - 1], last[0])
+
+
 ALL_PINS = [
     pin_golden_closed_form,
     pin_brute_force_decode,
@@ -488,4 +564,8 @@ ALL_PINS = [
     pin_int8_zero_row_and_slots,
     pin_int8_attention_brute_force,
     pin_int8_equals_bf16_path_on_exact_values,
+    pin_window_covering_all_is_full_attention,
+    pin_window_one_returns_last_v,
+    pin_window_equals_truncated_context,
+    pin_window_prefill_brute_force_and_last_row,
 ]

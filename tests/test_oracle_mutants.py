@@ -6,14 +6,14 @@ The mutants are compile-time variants of the C oracle (PKV_ORACLE_MUTANT):
 normaliser dropped, 7 token-major page layout, 8 cache-write slot off by one,
 9 scores taken against V, 10 merge weight sign flipped, 11 int8 code range
 128 instead of 127, 12 int8 rounding toward zero, 13 int8 V rows scaled by the
-K scale.
+K scale, 14 sliding window one key too wide.
 """
 import pytest
 
 import oracle
 import oracle_pins
 
-MUTANTS = list(range(1, 14))
+MUTANTS = list(range(1, 15))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
