@@ -159,6 +159,31 @@ pkv_status pkv_paged_attention_int8(void* out, const void* q, const void* k_cach
                                     size_t workspace_bytes, pkv_stream_t stream);
 
 /*
+ * paged_attention_window -- pkv_paged_attention under a sliding window: the
+ * query (position L_b - 1) attends only to its last `window` keys,
+ * max(0, L_b - window) .. L_b - 1.  The inference-lab page lists a
+ * sliding-window KV cache among its cache variants ("从零开始的LLM推理优化实
+ * 验室：从PyTorch基线到Triton内核的完整实践", section "KV缓存实验与长上下文
+ * 优化") without semantics; this is the reading taken.  Pages wholly before the
+ * window are never read; the first window page is masked row by row.
+ * window >= 1 (else PKV_ERR_INVALID_ARG); any context the block table holds.
+ *   workspace: >= pkv_paged_attention_window_workspace_size(...) bytes to let
+ *   the call split each window across CTAs, else one CTA per head group.
+ */
+pkv_status pkv_paged_attention_window(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache,
+                                      const int32_t* block_tables, int32_t MB,
+                                      const int32_t* context_lens, int32_t B,
+                                      int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                                      int32_t bs, float scale, int32_t window,
+                                      void* workspace, size_t workspace_bytes,
+                                      pkv_dtype dtype, pkv_stream_t stream);
+
+size_t pkv_paged_attention_window_workspace_size(int32_t B, int32_t Hq, int32_t Hkv,
+                                                 int32_t D, int32_t MB, int32_t bs,
+                                                 int32_t window);
+
+/*
  * paged_attention_split -- the split-KV ("flash-decoding") path with an
  * explicit split size.  Split c of sequence b covers logical pages
  * [c*pages_per_split, (c+1)*pages_per_split); each CTA writes its normalised

@@ -16,6 +16,7 @@ Calls (same names as the C ABI):
     kv_cache_write_int8(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping)
     paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables,
                          context_lens, scale, ...)
+    paged_attention_window(q, k_cache, v_cache, block_tables, context_lens, scale, window, ...)
 """
 from __future__ import annotations
 
@@ -54,6 +55,9 @@ EXPORTS = {
     "pkv_kv_cache_write_int8": ([_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
     "pkv_paged_attention_int8": ([_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32,
                                   _I32, _P, _SZ, _P], _I32),
+    "pkv_paged_attention_window": ([_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32,
+                                    _I32, _P, _SZ, _I32, _P], _I32),
+    "pkv_paged_attention_window_workspace_size": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "pkv_paged_attention_prefill": ([_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                      _I32, _I32, _I32, _F32, _I32, _P], _I32),
     "pkv_get_device_error": ([_P, ctypes.POINTER(_I32)], _I32),
@@ -220,6 +224,23 @@ def paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, co
                                       context_lens.data_ptr(), B, Hq, Hkv, D, NB, bs, float(scale),
                                       int(max_context_len), ws_ptr, ws_bytes, _stream(stream))
     _check(rc, "paged_attention_int8")
+    return out
+
+
+def paged_attention_window(q, k_cache, v_cache, block_tables, context_lens, scale: float, window: int,
+                           out=None, workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode where each query sees only its last ``window`` keys.  q [B, Hq, D] bf16."""
+    NB, Hkv, bs, D, B, Hq, MB, out = _decode_common(q, k_cache, v_cache, block_tables, context_lens, out)
+    lib = load_library()
+    need = int(lib.pkv_paged_attention_window_workspace_size(B, Hq, Hkv, D, MB, bs, int(window)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.pkv_paged_attention_window(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                        block_tables.data_ptr(), MB, context_lens.data_ptr(), B, Hq, Hkv, D, NB,
+                                        bs, float(scale), int(window), ws_ptr, ws_bytes, PKV_BF16, _stream(stream))
+    _check(rc, "paged_attention_window")
     return out
 
 

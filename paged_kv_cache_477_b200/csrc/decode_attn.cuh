@@ -61,8 +61,15 @@ struct DecodeParams {
   int32_t pages_per_split;
   int32_t num_splits;            // 1: write bf16 output directly
   int32_t cap_tokens;            // longest context this launch can hold
+  int32_t window;                // > 0: the query sees only its last `window` keys
   float scale_log2;              // scale * log2(e)
 };
+
+// First key a decode query (position L - 1) sees: 0, or L - window under a
+// sliding window of `window` keys (a query at p sees keys p - window < j <= p).
+__device__ __forceinline__ int window_first_key(int L, int window) {
+  return (window > 0 && L > window) ? L - window : 0;
+}
 
 // A ring stage holds PPS consecutive pages of one sequence: their K pages
 // side by side (ROWS = 16 * PPS contiguous key rows), then their V pages;
@@ -128,12 +135,13 @@ __device__ __forceinline__ void load_q(float2 (&q2)[HG][8], const __nv_bfloat16*
 }
 
 // ROWS key rows (K at kp, V at vp, row stride D) into the lane state.  Rows
-// r >= nvalid (past the end of the sequence or of the copied pages) take no
-// part in the max and are never read from V.
+// outside [nstart, nvalid) -- past the end of the sequence or of the copied
+// pages, or before a sliding window -- take no part in the max and are never
+// read from V.
 template <int D, int HG, int ROWS>
 __device__ __forceinline__ void attend_rows(LaneState<HG>& st, const float2 (&q2)[HG][8],
                                             const unsigned char* kp, const unsigned char* vp,
-                                            int nvalid, int rg, int ch0, int ch1) {
+                                            int nstart, int nvalid, int rg, int ch0, int ch1) {
   constexpr int LPR = D / 16, RPW = 32 / LPR, TPL = ROWS / RPW;
   float sc[TPL][HG];
 #pragma unroll
@@ -160,7 +168,7 @@ __device__ __forceinline__ void attend_rows(LaneState<HG>& st, const float2 (&q2
 
   bool valid[TPL];
 #pragma unroll
-  for (int t = 0; t < TPL; ++t) valid[t] = rg + t * RPW < nvalid;
+  for (int t = 0; t < TPL; ++t) valid[t] = rg + t * RPW < nvalid && rg + t * RPW >= nstart;
 
   float mp[HG];
   bool grow = false;
@@ -222,8 +230,8 @@ __device__ __forceinline__ void widen_i8x4(uint32_t w, float2& lo, float2& hi) {
 template <int D, int HG, int ROWS>
 __device__ __forceinline__ void attend_rows_i8(LaneState<HG>& st, const float2 (&q2)[HG][8],
                                                const unsigned char* kp, const unsigned char* vp,
-                                               const float* ksc, const float* vsc, int nvalid, int rg,
-                                               int sub) {
+                                               const float* ksc, const float* vsc, int nstart, int nvalid,
+                                               int rg, int sub) {
   constexpr int LPR = D / 16, RPW = 32 / LPR, TPL = ROWS / RPW;
   float sc[TPL][HG];
 #pragma unroll
@@ -254,8 +262,8 @@ __device__ __forceinline__ void attend_rows_i8(LaneState<HG>& st, const float2 (
 #pragma unroll
   for (int t = 0; t < TPL; ++t) {
     const int r = rg + t * RPW;
-    valid[t] = r < nvalid;
-    const float ks = valid[t] ? ksc[r] : 0.f;  // rows past the end are never read
+    valid[t] = r < nvalid && r >= nstart;
+    const float ks = valid[t] ? ksc[r] : 0.f;  // rows outside the range are never read
 #pragma unroll
     for (int h = 0; h < HG; ++h) sc[t][h] *= ks;
   }
@@ -401,7 +409,7 @@ __device__ __forceinline__ void drain_ring(uint32_t wbar, int issued) {
 // ============================================================================
 // One CTA per (split, head group, sequence).
 // ============================================================================
-template <int D, int HG, int NW, int SW, int PPS, bool I8 = false>
+template <int D, int HG, int NW, int SW, int PPS, bool I8 = false, bool WIN = false>
 __global__ void __launch_bounds__(NW * 32)
     decode_attn_kernel(const __grid_constant__ DecodeParams p) {
   using S = DecodeShape<D, HG, NW, SW, PPS, I8>;
@@ -412,7 +420,11 @@ __global__ void __launch_bounds__(NW * 32)
   const int head0 = kvh * p.G + (hsub % p.nsub) * HG;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int pg0 = split * p.pages_per_split;
+  int L = __ldg(p.context_lens + b);
+  // The sequence's pages from the first one its sliding window reaches (WIN;
+  // otherwise page 0, known before the length arrives); splits cut that range.
+  const int wp0 = WIN ? window_first_key(L < 0 ? 0 : min(L, p.cap_tokens), p.window) / kPageRows : 0;
+  const int pg0 = wp0 + split * p.pages_per_split;
   // The CTA's pages are cut into units of PPS consecutive pages, one unit per
   // ring stage; unit j of this warp is unit u = warp + j * NW, pages
   // pg0 + u * PPS + i.  Lane l of a chunk holds the block-table entries of
@@ -433,7 +445,6 @@ __global__ void __launch_bounds__(NW * 32)
     }
     return e;
   };
-  int L = __ldg(p.context_lens + b);
   const Entries raw0 = load_raw(0);
   Entries bt_nxt = load_raw(1);
   if (L < 0 || L > p.cap_tokens) {
@@ -532,6 +543,8 @@ __global__ void __launch_bounds__(NW * 32)
   // valid rows counted from this CTA's first page: the sequence's, and no
   // further than the CTA's own pages
   const int rows_cta = min(L - pg0 * kPageRows, n * kPageRows);
+  // rows before the window, counted the same way (<= 0 past the first split)
+  const int lo_cta = WIN ? window_first_key(L, p.window) - pg0 * kPageRows : 0;
   int done = 0;
   for (int j = 0; j < my_n; ++j, ++done) {
     const int s = j % SW;
@@ -544,10 +557,11 @@ __global__ void __launch_bounds__(NW * 32)
       attend_rows_i8<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES,
                                      reinterpret_cast<const float*>(kp + S::KS_OFF),
                                      reinterpret_cast<const float*>(kp + S::VS_OFF),
-                                     rows_cta - (warp + j * NW) * S::ROWS, rg, sub);
+                                     lo_cta - (warp + j * NW) * S::ROWS, rows_cta - (warp + j * NW) * S::ROWS, rg,
+                                     sub);
     else
-      attend_rows<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES, rows_cta - (warp + j * NW) * S::ROWS, rg,
-                                ch0, ch1);
+      attend_rows<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES, lo_cta - (warp + j * NW) * S::ROWS,
+                                  rows_cta - (warp + j * NW) * S::ROWS, rg, ch0, ch1);
     if (issued < my_n) {
       // the stage just read is refilled: order the generic-proxy reads of all
       // lanes before the copy engine's writes
@@ -585,7 +599,7 @@ struct MergeParams {
   const float* o_part;        // [B][Hq][C][D]
   const float* lse_part;      // [B][Hq][C]
   const int32_t* context_lens;
-  int32_t Hq, num_splits, pages_per_split, cap_tokens;
+  int32_t Hq, num_splits, pages_per_split, cap_tokens, window;
 };
 
 template <int D>
@@ -593,7 +607,7 @@ __global__ void __launch_bounds__(D) lse_merge_kernel(const __grid_constant__ Me
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   int L = __ldg(p.context_lens + b);
   L = L < 0 ? 0 : (L > p.cap_tokens ? p.cap_tokens : L);
-  const int npages = (L + kPageRows - 1) / kPageRows;
+  const int npages = (L + kPageRows - 1) / kPageRows - window_first_key(L, p.window) / kPageRows;
   const int nval = (npages + p.pages_per_split - 1) / p.pages_per_split;
   const size_t row = (size_t)b * p.Hq + h;
   const float* lse = p.lse_part + row * p.num_splits;

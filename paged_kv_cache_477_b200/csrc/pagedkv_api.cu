@@ -61,10 +61,10 @@ constexpr int stages_for(int D, bool I8) { return (I8 && D == 64) ? 6 : 3; }
 template <int D, int HG, bool I8 = false>
 using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D, I8), pages_per_stage(D, I8), I8>;
 
-template <int D, int HG, bool I8 = false>
+template <int D, int HG, bool I8 = false, bool WIN = false>
 struct DecodeKernel {
   static constexpr auto fn =
-      pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D, I8), pages_per_stage(D, I8), I8>;
+      pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D, I8), pages_per_stage(D, I8), I8, WIN>;
   // set the dynamic shared-memory limit once per device; return CTAs per SM
   static int prepare(int dev) {
     static int occ[kMaxDevices] = {0};
@@ -154,25 +154,26 @@ DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, 
   return pl;
 }
 
-template <int D, int HG, bool I8 = false>
+template <int D, int HG, bool I8 = false, bool WIN = false>
 pkv_status launch_decode_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C,
                            cudaStream_t st) {
-  if (DecodeKernel<D, HG, I8>::prepare(current_device()) < 0) return PKV_ERR_CUDA;
+  using K = DecodeKernel<D, HG, I8, WIN>;
+  if (K::prepare(current_device()) < 0) return PKV_ERR_CUDA;
   dim3 grid(C, Hkv * nsub, B);
-  DecodeKernel<D, HG, I8>::fn<<<grid, DecodeS<D, HG, I8>::THREADS, DecodeS<D, HG, I8>::SMEM_BYTES, st>>>(p);
+  K::fn<<<grid, DecodeS<D, HG, I8>::THREADS, DecodeS<D, HG, I8>::SMEM_BYTES, st>>>(p);
   return launch_status();
 }
 
-template <bool I8>
+template <bool I8, bool WIN = false>
 pkv_status launch_decode_any(const pkv::DecodeParams& p, int D, int HG, int B, int Hkv, int nsub, int C,
                              cudaStream_t st) {
   if (D == 128)
-    return HG == 4 ? launch_decode_t<128, 4, I8>(p, B, Hkv, nsub, C, st)
-           : HG == 2 ? launch_decode_t<128, 2, I8>(p, B, Hkv, nsub, C, st)
-                     : launch_decode_t<128, 1, I8>(p, B, Hkv, nsub, C, st);
-  return HG == 4 ? launch_decode_t<64, 4, I8>(p, B, Hkv, nsub, C, st)
-         : HG == 2 ? launch_decode_t<64, 2, I8>(p, B, Hkv, nsub, C, st)
-                   : launch_decode_t<64, 1, I8>(p, B, Hkv, nsub, C, st);
+    return HG == 4 ? launch_decode_t<128, 4, I8, WIN>(p, B, Hkv, nsub, C, st)
+           : HG == 2 ? launch_decode_t<128, 2, I8, WIN>(p, B, Hkv, nsub, C, st)
+                     : launch_decode_t<128, 1, I8, WIN>(p, B, Hkv, nsub, C, st);
+  return HG == 4 ? launch_decode_t<64, 4, I8, WIN>(p, B, Hkv, nsub, C, st)
+         : HG == 2 ? launch_decode_t<64, 2, I8, WIN>(p, B, Hkv, nsub, C, st)
+                   : launch_decode_t<64, 1, I8, WIN>(p, B, Hkv, nsub, C, st);
 }
 
 template <int D>
@@ -203,7 +204,7 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
                       const int32_t* block_tables, int32_t MB, const int32_t* context_lens,
                       int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB, float scale,
                       const DecodePlan& pl, void* workspace, cudaStream_t st,
-                      const float* k_scale = nullptr, const float* v_scale = nullptr) {
+                      const float* k_scale = nullptr, const float* v_scale = nullptr, int32_t window = 0) {
   const int G = Hq / Hkv, HG = heads_per_cta(G), nsub = G / HG;
   const int C = pl.num_splits;
   pkv::DecodeParams p{};
@@ -221,14 +222,18 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
   p.num_splits = C;
   p.cap_tokens = (int32_t)std::min<int64_t>((int64_t)MB, (int64_t)C * pl.pages_per_split) * pkv::kPageRows;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.window = window;
+  // a window bounds the pages read, not the context: any length the table holds
+  if (window > 0) p.cap_tokens = MB * pkv::kPageRows;
   if (C > 1) {
     const size_t rows = (size_t)B * Hq * C;
     p.o_part = static_cast<float*>(workspace);
     p.lse_part = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) +
                                           round256(rows * D * sizeof(float)));
   }
-  pkv_status s = k_scale ? launch_decode_any<true>(p, D, HG, B, Hkv, nsub, C, st)
-                         : launch_decode_any<false>(p, D, HG, B, Hkv, nsub, C, st);
+  pkv_status s = k_scale    ? launch_decode_any<true>(p, D, HG, B, Hkv, nsub, C, st)
+                 : window > 0 ? launch_decode_any<false, true>(p, D, HG, B, Hkv, nsub, C, st)
+                              : launch_decode_any<false>(p, D, HG, B, Hkv, nsub, C, st);
   if (s != PKV_OK) return s;
   int launches = 1;
   if (C > 1) {
@@ -241,6 +246,7 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
     mp.num_splits = C;
     mp.pages_per_split = pl.pages_per_split;
     mp.cap_tokens = p.cap_tokens;
+    mp.window = window;
     s = D == 128 ? launch_merge_t<128>(mp, B, Hq, st) : launch_merge_t<64>(mp, B, Hq, st);
     if (s != PKV_OK) return s;
     ++launches;
@@ -429,6 +435,38 @@ pkv_status pkv_paged_attention_int8(void* out, const void* q, const void* k_cach
   return run_decode(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq, Hkv, D, NB, scale, pl,
                     workspace, static_cast<cudaStream_t>(stream), k_scale ? k_scale : kNoScale,
                     v_scale ? v_scale : kNoScale);
+}
+
+// pages a window of W keys can touch: W keys starting anywhere in a page
+int window_pages(int32_t window) { return (int)(((int64_t)window + pkv::kPageRows - 2) / pkv::kPageRows) + 1; }
+
+pkv_status pkv_paged_attention_window(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, int32_t MB, const int32_t* context_lens,
+                                      int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB, int32_t bs,
+                                      float scale, int32_t window, void* workspace, size_t workspace_bytes,
+                                      pkv_dtype dtype, pkv_stream_t stream) {
+  t_launches = 0;
+  pkv_status s = check_decode_args(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq,
+                                    Hkv, D, NB, bs, dtype);
+  if (s != PKV_OK || B == 0) return s;
+  if (window < 1) return PKV_ERR_INVALID_ARG;
+  // plan over the pages a window touches; the kernel starts each sequence at
+  // the first page its window reaches
+  const int32_t span = (int32_t)std::min<int64_t>((int64_t)window_pages(window) * bs, (int64_t)MB * bs);
+  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, span);
+  if (pl.num_splits > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned16(workspace)))
+    pl = DecodePlan{1, std::max<int32_t>(MB, 1), 0};  // no room: one CTA per head group
+  if (pl.num_splits == 1) pl.pages_per_split = std::max<int32_t>(MB, 1);
+  return run_decode(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq, Hkv, D, NB, scale, pl,
+                    workspace, static_cast<cudaStream_t>(stream), nullptr, nullptr, window);
+}
+
+size_t pkv_paged_attention_window_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB,
+                                                 int32_t bs, int32_t window) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || (D != 64 && D != 128) || bs != pkv::kPageRows || window < 1)
+    return 0;
+  const int32_t span = (int32_t)std::min<int64_t>((int64_t)window_pages(window) * bs, (int64_t)MB * bs);
+  return plan_auto(B, Hq, Hkv, D, MB, bs, span).workspace;
 }
 
 size_t pkv_split_workspace_size(int32_t B, int32_t Hq, int32_t D, int32_t num_splits) {

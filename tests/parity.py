@@ -74,6 +74,12 @@ class HostCase:
                                             np.ascontiguousarray(self.bt[rows]),
                                             np.ascontiguousarray(self.lens[rows]), self.case.scale)
 
+    def decode_window_ref(self, window, rows=None):
+        rows = np.arange(self.case.B) if rows is None else np.asarray(rows)
+        return oracle.get().paged_attention_window(np.ascontiguousarray(self.q[rows]), self.k, self.v,
+                                                   np.ascontiguousarray(self.bt[rows]),
+                                                   np.ascontiguousarray(self.lens[rows]), self.case.scale, window)
+
     def prefill_ref(self, seqs=None):
         """Reference for whole sequences ``seqs``; returns (ref, token_index)."""
         c = self.case

@@ -235,3 +235,40 @@ def test_decode_ragged_batch_auto_and_split_agree():
     assert pkv.last_launch_count() == 2
     assert_close(split, ref, "split pps=64")
     _no_device_error()
+
+
+# --------------------------------------------------------------------------- #
+# sliding window                                                               #
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("window", [1, 15, 16, 17, 100, 1000])
+def test_decode_window_edges(D, window):
+    """Windows shorter and longer than the contexts, starting inside a page
+    and on a page boundary; canaries in every slot outside the contexts."""
+    case = _decode_case(EDGE_LENS, 8, 2, D, seed=300 + D + window)
+    out = pkv.paged_attention_window(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                     case.context_lens, case.scale, window)
+    assert_close(out, HostCase(case).decode_window_ref(window), f"window={window} D={D}")
+    assert torch.count_nonzero(out[0]) == 0              # empty context -> zero row
+    _no_device_error()
+
+
+@pytest.mark.parametrize("window", [64, 500, 4096])
+def test_decode_window_long_contexts_split(window):
+    """Contexts far longer than the window: only the window's pages are read,
+    split across CTAs when the window is long."""
+    case = _decode_case([20000, 3, 5000, 777, 4096, 12345], 32, 8, 128, seed=310 + window)
+    out = pkv.paged_attention_window(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                     case.context_lens, case.scale, window)
+    if window == 4096:                                   # 257 window pages: split
+        assert pkv.last_launch_count() == 2
+    assert_close(out, HostCase(case).decode_window_ref(window), f"window={window}")
+    _no_device_error()
+
+
+def test_decode_window_rejects_zero():
+    case = _decode_case([40], 4, 2, 64, seed=320)
+    with pytest.raises(pkv.PagedKVError):
+        pkv.paged_attention_window(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                   case.context_lens, case.scale, 0)
