@@ -269,6 +269,20 @@ pkv_status pkv_paged_attention_prefill(
     int32_t bs, float scale, pkv_dtype dtype, pkv_stream_t stream);
 
 /*
+ * paged_attention_prefill_window -- pkv_paged_attention_prefill under a
+ * sliding window: query i of sequence b (position p = L_b - Q_b + i) sees
+ * keys max(0, p - window + 1) .. p (the reading of the inference-lab page's
+ * sliding-window cache, as for pkv_paged_attention_window).  Key tiles below
+ * every row's window are skipped; edge tiles are masked per row.  window >= 1.
+ */
+pkv_status pkv_paged_attention_prefill_window(
+    void* out, const void* q, const int32_t* query_start_loc,
+    const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    int32_t MB, const int32_t* context_lens, int32_t B, int32_t sumQ,
+    int32_t max_q_len, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+    int32_t bs, float scale, int32_t window, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error
  * word (0 = none, else a pkv_status value recorded by a kernel).
  */

@@ -17,6 +17,8 @@ Calls (same names as the C ABI):
     paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables,
                          context_lens, scale, ...)
     paged_attention_window(q, k_cache, v_cache, block_tables, context_lens, scale, window, ...)
+    paged_attention_prefill_window(q, query_start_loc, k_cache, v_cache, block_tables,
+                                   context_lens, scale, max_q_len, window, ...)
 """
 from __future__ import annotations
 
@@ -60,6 +62,8 @@ EXPORTS = {
     "pkv_paged_attention_window_workspace_size": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
     "pkv_paged_attention_prefill": ([_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                      _I32, _I32, _I32, _F32, _I32, _P], _I32),
+    "pkv_paged_attention_prefill_window": ([_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
+                                            _I32, _I32, _I32, _F32, _I32, _I32, _P], _I32),
     "pkv_get_device_error": ([_P, ctypes.POINTER(_I32)], _I32),
     "pkv_last_launch_count": ([], _I32),
     "pkv_status_string": ([_I32], ctypes.c_char_p),
@@ -341,6 +345,30 @@ def paged_attention_prefill(q, query_start_loc, k_cache, v_cache, block_tables, 
         v_cache.data_ptr(), block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
         B, sumQ, int(max_q_len), Hq, Hkv, D, NB, bs, float(scale), PKV_BF16, _stream(stream))
     _check(rc, "paged_attention_prefill")
+    return out
+
+
+def paged_attention_prefill_window(q, query_start_loc, k_cache, v_cache, block_tables, context_lens,
+                                   scale: float, max_q_len: int, window: int, out=None, stream=None) -> torch.Tensor:
+    """Causal chunked prefill where a query at position p sees keys p - window < j <= p."""
+    NB, Hkv, bs, D = _cache_dims(k_cache, v_cache)
+    _contig(_dev(q, "q", torch.bfloat16), "q")
+    _contig(_dev(query_start_loc, "query_start_loc", torch.int32), "query_start_loc")
+    _contig(_dev(block_tables, "block_tables", torch.int32), "block_tables")
+    _contig(_dev(context_lens, "context_lens", torch.int32), "context_lens")
+    sumQ, Hq, Dq = q.shape
+    B = context_lens.numel()
+    if Dq != D or query_start_loc.numel() != B + 1 or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch between q, query_start_loc, block_tables, context_lens")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _contig(_dev(out, "out", torch.bfloat16), "out")
+    rc = load_library().pkv_paged_attention_prefill_window(
+        out.data_ptr(), q.data_ptr(), query_start_loc.data_ptr(), k_cache.data_ptr(),
+        v_cache.data_ptr(), block_tables.data_ptr(), block_tables.shape[1], context_lens.data_ptr(),
+        B, sumQ, int(max_q_len), Hq, Hkv, D, NB, bs, float(scale), int(window), PKV_BF16, _stream(stream))
+    _check(rc, "paged_attention_prefill_window")
     return out
 
 

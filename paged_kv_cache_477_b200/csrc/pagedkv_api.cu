@@ -292,14 +292,15 @@ int prefill_prepare(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return -1;
   std::lock_guard<std::mutex> g(mu);
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(pkv::prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pkv::pf::SMEM_BYTES) != cudaSuccess)
-      return -1;
-    // the kernel's setmaxnreg split is sized for exactly this register count
-    cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, pkv::prefill_attn_kernel) != cudaSuccess ||
-        attr.numRegs != pkv::pf::REGS_LAUNCH)
-      return -2;
+    for (const void* fn : {reinterpret_cast<const void*>(pkv::prefill_attn_kernel<false>),
+                           reinterpret_cast<const void*>(pkv::prefill_attn_kernel<true>)}) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pkv::pf::SMEM_BYTES) !=
+          cudaSuccess)
+        return -1;
+      // the kernel's setmaxnreg split is sized for exactly this register count
+      cudaFuncAttributes attr;
+      if (cudaFuncGetAttributes(&attr, fn) != cudaSuccess || attr.numRegs != pkv::pf::REGS_LAUNCH) return -2;
+    }
     done[dev] = 1;
   }
   return 0;
@@ -523,13 +524,14 @@ pkv_status pkv_paged_attention_split(void* out, const void* q, const void* k_cac
                     scale, pl, workspace, static_cast<cudaStream_t>(stream));
 }
 
-pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* query_start_loc,
-                                       const void* k_cache, const void* v_cache,
-                                       const int32_t* block_tables, int32_t MB,
-                                       const int32_t* context_lens, int32_t B, int32_t sumQ,
-                                       int32_t max_q_len, int32_t Hq, int32_t Hkv, int32_t D,
-                                       int32_t NB, int32_t bs, float scale, pkv_dtype dtype,
-                                       pkv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+pkv_status prefill_impl(void* out, const void* q, const int32_t* query_start_loc, const void* k_cache,
+                        const void* v_cache, const int32_t* block_tables, int32_t MB,
+                        const int32_t* context_lens, int32_t B, int32_t sumQ, int32_t max_q_len, int32_t Hq,
+                        int32_t Hkv, int32_t D, int32_t NB, int32_t bs, float scale, int32_t window,
+                        pkv_dtype dtype, pkv_stream_t stream) {
   t_launches = 0;
   if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
   if (B < 0 || sumQ < 0 || max_q_len < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || NB < 0 || MB < 0 || bs <= 0)
@@ -578,12 +580,46 @@ pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* 
   const int nct = (max_q_len + ppc - 1) / ppc;
   if (nct > 65535 || B > 65535) return PKV_ERR_UNSUPPORTED;
   p.nct = nct;
+  p.window = window;
   dim3 grid(Hkv, B, nct);
-  pkv::prefill_attn_kernel<<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(
-      p, tm_q, tm_k, tm_v);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (window > 0)
+    pkv::prefill_attn_kernel<true><<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, st>>>(p, tm_q, tm_k, tm_v);
+  else
+    pkv::prefill_attn_kernel<false><<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, st>>>(p, tm_q, tm_k, tm_v);
   pkv_status s = launch_status();
   if (s == PKV_OK) t_launches = 1;
   return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+pkv_status pkv_paged_attention_prefill(void* out, const void* q, const int32_t* query_start_loc,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* block_tables, int32_t MB,
+                                       const int32_t* context_lens, int32_t B, int32_t sumQ,
+                                       int32_t max_q_len, int32_t Hq, int32_t Hkv, int32_t D,
+                                       int32_t NB, int32_t bs, float scale, pkv_dtype dtype,
+                                       pkv_stream_t stream) {
+  return prefill_impl(out, q, query_start_loc, k_cache, v_cache, block_tables, MB, context_lens, B, sumQ,
+                      max_q_len, Hq, Hkv, D, NB, bs, scale, 0, dtype, stream);
+}
+
+pkv_status pkv_paged_attention_prefill_window(void* out, const void* q, const int32_t* query_start_loc,
+                                              const void* k_cache, const void* v_cache,
+                                              const int32_t* block_tables, int32_t MB,
+                                              const int32_t* context_lens, int32_t B, int32_t sumQ,
+                                              int32_t max_q_len, int32_t Hq, int32_t Hkv, int32_t D,
+                                              int32_t NB, int32_t bs, float scale, int32_t window,
+                                              pkv_dtype dtype, pkv_stream_t stream) {
+  if (window < 1) {
+    t_launches = 0;
+    return PKV_ERR_INVALID_ARG;
+  }
+  return prefill_impl(out, q, query_start_loc, k_cache, v_cache, block_tables, MB, context_lens, B, sumQ,
+                      max_q_len, Hq, Hkv, D, NB, bs, scale, window, dtype, stream);
 }
 
 pkv_status pkv_get_device_error(pkv_stream_t stream, int32_t* err_out) {

@@ -51,6 +51,7 @@ struct PrefillParams {
   const int32_t* context_lens;     // [B]
   int32_t B, Hq, Hkv, NB, MB, G, sumQ;
   int32_t nct;                     // tasks (query-tile pairs) per (sequence, kv head)
+  int32_t window;                  // > 0: a query at p sees only keys p - window < j <= p
   float scale_log2;                // scale * log2(e), >= 0
 };
 
@@ -128,14 +129,16 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 }
 
 // Task t of a launch: query-tile pair ct of sequence b, kv head kvh, in grid
-// order (kv head fastest, then sequence, then the pairs last first).  n is
-// the number of 128-key tiles its rows see (0: nothing to do).  Each role of
+// order (kv head fastest, then sequence, then the pairs last first).  Its
+// rows see key tiles [j0, n) (n = 0: nothing to do; j0 > 0 only under a
+// sliding window, where the earliest row's window starts).  Each role of
 // the CTA computes it for itself (three cached loads) instead of keeping it
 // live across the register split.
 struct PrefillTask {
-  int b, kvh, ct, qs, Qb, L, p0, n;
+  int b, kvh, ct, qs, Qb, L, p0, n, j0;
 };
 
+template <bool WIN>
 __device__ __forceinline__ PrefillTask prefill_task(const PrefillParams& p, int t) {
   PrefillTask k;
   const int per = p.B * p.Hkv;
@@ -147,16 +150,24 @@ __device__ __forceinline__ PrefillTask prefill_task(const PrefillParams& p, int 
   k.L = __ldg(p.context_lens + k.b);
   k.p0 = k.ct * pf::NQT * (pf::BM / p.G);
   k.n = 0;
+  k.j0 = 0;
   if (k.Qb < 0 || k.L < k.Qb || k.L > p.MB * 16 || k.qs < 0 || k.qs + k.Qb > p.sumQ) {
     set_error(PKV_ERR_BOUNDS);
   } else if (k.p0 < k.Qb) {
     const int last_pos = min(k.p0 + pf::NQT * (pf::BM / p.G), k.Qb) - 1;
     const int kv_end = k.L - k.Qb + last_pos + 1;  // keys the last valid row can see
     k.n = (kv_end + pf::BN - 1) / pf::BN;
+    if (WIN) {
+      const int first_key = k.L - k.Qb + k.p0 - p.window + 1;  // the first row's window start
+      k.j0 = first_key > 0 ? first_key / pf::BN : 0;
+    }
   }
   return k;
 }
 
+// WIN: sliding window of p.window keys (a separate instantiation, so the
+// plain causal kernel carries none of its per-row bounds).
+template <bool WIN>
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -172,7 +183,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   __shared__ int s_flag;
   if (threadIdx.x == 0) {
     int f = *reinterpret_cast<volatile int*>(&g_error_word) == PKV_ERR_TIMEOUT;
-    f |= prefill_task(p, t).n == 0;  // nothing to do (or bad lengths, reported)
+    f |= prefill_task<WIN>(p, t).n == 0;  // nothing to do (or bad lengths, reported)
     s_flag = f;
   }
   __syncthreads();
@@ -219,7 +230,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         tc::prefetch_tensormap(&tm_k);
         tc::prefetch_tensormap(&tm_v);
       }
-      const PrefillTask k = prefill_task(p, t);
+      const PrefillTask k = prefill_task<WIN>(p, t);
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(pf::B_Q), pf::NQT * pf::TILE_BYTES);
         for (int i = 0; i < pf::NQT; ++i) {
@@ -233,7 +244,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       const int npages = (k.L + 15) / 16;
       int issued_k = 0, issued_v = 0;
       bool ok = true;
-      for (int j = 0; j < k.n; ++j) {
+      for (int j = k.j0; j < k.n; ++j) {
+        const int jl = j - k.j0;  // position in this task's key-tile stream
         int blk = p.NB;  // out of range: TMA fills the page with zeros
         if (lane < 8) {
           const int pg = j * 8 + lane;
@@ -246,9 +258,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           }
         }
         // K tile j
-        const int ks = j % pf::KSTAGES;
+        const int ks = jl % pf::KSTAGES;
         if (lane == 0) {
-          if (j >= pf::KSTAGES) ok = mbar_wait(bar(pf::B_KEMPTY + ks), ((j / pf::KSTAGES) - 1) & 1);
+          if (jl >= pf::KSTAGES) ok = mbar_wait(bar(pf::B_KEMPTY + ks), ((jl / pf::KSTAGES) - 1) & 1);
           if (ok) mbar_arrive_expect_tx(bar(pf::B_KFULL + ks), pf::TILE_BYTES);
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -259,9 +271,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         }
         ++issued_k;
         // V tile j
-        const int vs = j % pf::VSTAGES;
+        const int vs = jl % pf::VSTAGES;
         if (lane == 0) {
-          if (j >= pf::VSTAGES) ok = mbar_wait(bar(pf::B_VEMPTY + vs), ((j / pf::VSTAGES) - 1) & 1);
+          if (jl >= pf::VSTAGES) ok = mbar_wait(bar(pf::B_VEMPTY + vs), ((jl / pf::VSTAGES) - 1) & 1);
           if (ok) mbar_arrive_expect_tx(bar(pf::B_VFULL + vs), pf::TILE_BYTES);
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -309,10 +321,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         tc::commit(bar(pf::B_SFULL + i));
         if (i == pf::NQT - 1) tc::commit(bar(pf::B_KEMPTY + ks));
       };
-      // O_i += P_i V for V tile tv = key tile j
-      auto pv = [&](int i, int j, int tail_rows, int tail_page) -> bool {
+      // O_i += P_i V for V tile tv = key tile j, the task's jl-th
+      auto pv = [&](int i, int jl, int j, int tail_rows, int tail_page) -> bool {
         const int vs = tv % pf::VSTAGES;
-        if (!mbar_wait(bar(pf::B_PFULL + i), j & 1)) return false;
+        if (!mbar_wait(bar(pf::B_PFULL + i), jl & 1)) return false;
         if (i == 0) {
           if (!mbar_wait(bar(pf::B_VFULL + vs), (tv / pf::VSTAGES) & 1)) return false;
           if (tail_rows != 0 && tail_page / 8 == j) {
@@ -334,7 +346,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         const uint32_t d_o = p_t + pf::O_COL;
 #pragma unroll
         for (int kk = 0; kk < pf::BN / 16; ++kk)
-          tc::mma_ts(d_o, p_t + kk * 8, dv + kk * (2048 >> 4), IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(d_o, p_t + kk * 8, dv + kk * (2048 >> 4), IDESC_PV, (jl > 0 || kk > 0) ? 1u : 0u);
         tc::commit(bar(pf::B_OREADY + i));
         if (i == pf::NQT - 1) {
           tc::commit(bar(pf::B_VEMPTY + vs));
@@ -343,7 +355,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         return true;
       };
 
-      const PrefillTask k = prefill_task(p, t);
+      const PrefillTask k = prefill_task<WIN>(p, t);
       // the page holding the sequence's last key, if it is only partly valid
       const int tail_rows = k.L % 16, tail_page = (k.L - 1) / 16;
       bool ok = mbar_wait(bar(pf::B_Q), 0);
@@ -353,9 +365,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         for (int i = 0; i < pf::NQT; ++i) qk(i);
         ++tk;
       }
-      for (int j = 1; j < k.n && ok; ++j) {
+      const int nl = k.n - k.j0;  // key tiles of this task
+      for (int jl = 1; jl < nl && ok; ++jl) {
         for (int i = 0; i < pf::NQT && ok; ++i) {
-          ok = pv(i, j - 1, tail_rows, tail_page);  // frees query tile i's score buffer (P_{j-1} is read first)
+          ok = pv(i, jl - 1, k.j0 + jl - 1, tail_rows, tail_page);  // frees query tile i's score buffer
           if (ok && i == 0) ok = mbar_wait(bar(pf::B_KFULL + tk % pf::KSTAGES), (tk / pf::KSTAGES) & 1);
           if (ok) {
             tc::fence_after_sync();
@@ -364,7 +377,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         }
         ++tk;
       }
-      for (int i = 0; i < pf::NQT && ok; ++i) ok = pv(i, k.n - 1, tail_rows, tail_page);
+      for (int i = 0; i < pf::NQT && ok; ++i) ok = pv(i, nl - 1, k.n - 1, tail_rows, tail_page);
       // all MMAs of this CTA retired before TMEM is released
       tc::commit(bar(pf::B_MMADONE));
       mbar_wait(bar(pf::B_MMADONE), 0);
@@ -379,15 +392,17 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     const uint32_t s_addr = tmem + lane_off + qt * pf::TILE_COLS;
     const uint32_t o_addr = s_addr + pf::O_COL;
     const float sl2 = p.scale_log2;
-    const PrefillTask k = prefill_task(p, t);
+    const PrefillTask k = prefill_task<WIN>(p, t);
     const int pos = k.p0 + qt * PPT + r / G, hh = r % G;
     const bool row_valid = pos < k.Qb;
     const int limit = k.L - k.Qb + min(pos, k.Qb - 1);  // last key this row may see
+    const int lo = WIN ? limit - p.window + 1 : 0;  // first key this row may see
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     {  // key tiles, then the epilogue
-      for (int j = 0; j < k.n; ++j) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_SFULL + qt), j & 1))) {
+      for (int j = k.j0; j < k.n; ++j) {
+        const int jl = j - k.j0;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_SFULL + qt), jl & 1))) {
           ok = false;
           break;
         }
@@ -397,11 +412,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         for (int c = 0; c < pf::BN; c += 32) tc::ld_32x32b_x32(s_addr + c, sr + c);
         tc::wait_ld();
         const int kv0 = j * pf::BN;
-        const bool diag = kv0 + pf::BN - 1 > limit;
+        // edge tiles: the causal diagonal, or (sliding window) the row's window start
+        const bool diag = kv0 + pf::BN - 1 > limit || (WIN && kv0 < lo);
         if (diag) {
 #pragma unroll
           for (int c = 0; c < pf::BN; ++c)
-            if (kv0 + c > limit) sr[c] = __float_as_uint(-INFINITY);
+            if (kv0 + c > limit || (WIN && kv0 + c < lo)) sr[c] = __float_as_uint(-INFINITY);
         }
         // row max: eight independent chains of three-input maxima
         float mxk[8];
@@ -421,9 +437,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           // warp-uniform branch: the TMEM accesses below are warp-collective;
           // rows that keep their max use alpha = 1
           const float alpha = grow ? ex2(m_run - m_tile) : 1.f;  // 0 on the first tile
-          if (j > 0) {
+          if (jl > 0) {
             // O holds P.V of earlier tiles: rescale it once the last of them is done
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (j - 1) & 1))) {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (jl - 1) & 1))) {
               ok = false;
               break;
             }
@@ -460,8 +476,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                             ? exp2_poly2(x)
                             : make_float2(ex2(x.x), ex2(x.y));
             if (diag) {  // masked keys: exactly 0 (the polynomial, or a zero scale, would not give it)
-              if (kv0 + c > limit) pr.x = 0.f;
-              if (kv0 + c + 1 > limit) pr.y = 0.f;
+              if (kv0 + c > limit || (WIN && kv0 + c < lo)) pr.x = 0.f;
+              if (kv0 + c + 1 > limit || (WIN && kv0 + c + 1 < lo)) pr.y = 0.f;
             }
             rs[(c / 2) & 3] = __fadd2_rn(rs[(c / 2) & 3], pr);
             __nv_bfloat162 h2 = __floats2bfloat162_rn(pr.x, pr.y);
@@ -477,7 +493,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(pf::B_PFULL + qt));
       }
-      if (ok && __all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (k.n - 1) & 1))) {
+      if (ok && __all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (k.n - k.j0 - 1) & 1))) {
         tc::fence_after_sync();
         uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)(k.qs + pos) * p.Hq + k.kvh * G + hh) * pf::D);
         // O / l to global memory

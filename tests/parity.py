@@ -80,14 +80,20 @@ class HostCase:
                                                    np.ascontiguousarray(self.bt[rows]),
                                                    np.ascontiguousarray(self.lens[rows]), self.case.scale, window)
 
-    def prefill_ref(self, seqs=None):
-        """Reference for whole sequences ``seqs``; returns (ref, token_index)."""
+    def prefill_ref(self, seqs=None, window=0):
+        """Reference for whole sequences ``seqs`` (sliding ``window`` if > 0);
+        returns (ref, token_index)."""
         c = self.case
         seqs = list(range(c.B)) if seqs is None else list(seqs)
         qsl = self.qsl
         tok = np.concatenate([np.arange(qsl[b], qsl[b + 1]) for b in seqs]).astype(np.int64)
         sub_qsl = np.concatenate([[0], np.cumsum([qsl[b + 1] - qsl[b] for b in seqs])]).astype(np.int32)
-        ref = oracle.get().paged_attention_prefill(np.ascontiguousarray(self.q[tok]), sub_qsl, self.k, self.v,
-                                                   np.ascontiguousarray(self.bt[seqs]),
-                                                   np.ascontiguousarray(self.lens[seqs]), c.scale)
+        if window:
+            ref = oracle.get().paged_attention_prefill_window(np.ascontiguousarray(self.q[tok]), sub_qsl, self.k,
+                                                              self.v, np.ascontiguousarray(self.bt[seqs]),
+                                                              np.ascontiguousarray(self.lens[seqs]), c.scale, window)
+        else:
+            ref = oracle.get().paged_attention_prefill(np.ascontiguousarray(self.q[tok]), sub_qsl, self.k, self.v,
+                                                       np.ascontiguousarray(self.bt[seqs]),
+                                                       np.ascontiguousarray(self.lens[seqs]), c.scale)
         return ref, tok

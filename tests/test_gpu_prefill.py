@@ -116,3 +116,23 @@ def test_prefill_zero_scale_gives_mean_of_visible_values():
     ref, tok = host.prefill_ref()
     assert_close(out[tok], ref, "prefill scale=0")
     assert pkv.get_device_error() == 0
+
+
+@pytest.mark.parametrize("window", [1, 17, 128, 129, 300, 5000])
+def test_prefill_window(window):
+    """Sliding window: tiles below every row's window skipped, edge tiles masked
+    per row (windows shorter than a tile, tile-aligned, spanning tiles, wider
+    than the context)."""
+    lens = [700, 77, 1300, 45]
+    qlens = [300, 77, 129, 1]
+    case = _prefill_case(lens, qlens, 16, 4, seed=560 + window)
+    host = HostCase(case)
+    pkv.kv_cache_write(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping)
+    out = pkv.paged_attention_prefill_window(case.q, case.query_start_loc, case.k_cache, case.v_cache,
+                                             case.block_tables, case.context_lens, case.scale, case.max_q_len,
+                                             window)
+    assert pkv.last_launch_count() == 1
+    host.apply_write()
+    ref, tok = host.prefill_ref(window=window)
+    assert_close(out[tok], ref, f"prefill window={window}")
+    assert pkv.get_device_error() == 0
