@@ -323,6 +323,25 @@ def extras(peaks):
                      "l2": "inputs larger than L2"}
         del c, out, ws
         torch.cuda.empty_cache()
+    # sliding window of 1024 keys over the Llama-3-8B-shaped batch (ctx 4096)
+    c = wl.workload(WORKLOAD, device="cuda")
+    out = torch.empty_like(c.q)
+    W = 1024
+    ws = torch.empty(max(1, pkv.window_workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, W)), dtype=torch.uint8,
+                     device="cuda")
+    fn = lambda: pkv.paged_attention_window(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale,
+                                            W, out=out, workspace=ws)
+    time_calls(fn, 3)
+    ms = statistics.median(time_calls(fn, 20))
+    wbytes = sum(min(L, W) for L in c.lens) * c.Hkv * c.D * 2 * 2 + 2 * c.B * c.Hq * c.D * 2 + \
+        sum(-(-min(L, W) // 16) for L in c.lens) * 4 + c.B * 4
+    gbs = wbytes / (ms * 1e-3) / 1e9
+    res["llama3_8b_decode_window1024"] = {"GB/s": round(gbs, 1), "us": round(ms * 1e3, 2),
+                                          "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                                          "launches": pkv.last_launch_count(), "bytes": wbytes,
+                                          "l2": "window pages of 128 x 8 heads: 512 MiB, larger than L2"}
+    del c, out, ws
+    torch.cuda.empty_cache()
     # INT8 cache (one fp32 scale per row): same shape as the headline step
     c = wl.workload("llama3_8b_decode_int8", device="cuda")
     pkv.kv_cache_write_int8(c.new_key, c.new_value, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.slot_mapping)

@@ -248,6 +248,10 @@ def paged_attention_window(q, k_cache, v_cache, block_tables, context_lens, scal
     return out
 
 
+def window_workspace_size(B, Hq, Hkv, D, MB, bs, window) -> int:
+    return int(load_library().pkv_paged_attention_window_workspace_size(B, Hq, Hkv, D, MB, bs, int(window)))
+
+
 def workspace_size(B, Hq, Hkv, D, MB, bs=16, max_context_len: int = 0) -> int:
     return int(load_library().pkv_paged_attention_workspace_size(B, Hq, Hkv, D, MB, bs, max_context_len))
 
