@@ -88,6 +88,11 @@ class Oracle:
                                                    _I32, _F32, _I32]
         lib.ref_paged_attention_prefill_window.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
                                                            _I32, _I32, _I32, _F32, _I32]
+        lib.ref_rope_rows.argtypes = [_P, _P, _I64, _P, _I64, _I32, _I32, ctypes.c_double]
+        lib.ref_kv_cache_write_rope.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                                ctypes.c_double]
+        lib.ref_rope_rows.restype = ctypes.c_int
+        lib.ref_kv_cache_write_rope.restype = ctypes.c_int
         for f in ("ref_kv_cache_write", "ref_paged_attention", "ref_contiguous_attention",
                   "ref_paged_attention_prefill", "ref_decode_partials", "ref_lse_merge",
                   "ref_kv_cache_write_int8", "ref_paged_attention_int8", "ref_paged_attention_window",
@@ -150,6 +155,32 @@ class Oracle:
                                                MB, _ptr(context_lens), B, Hq, Hkv, D, NB, bs, float(scale))
         self._check(rc, "paged_attention_int8", allow_bounds)
         return out
+
+    # -- rotary position embedding ------------------------------------------
+    def rope_rows(self, x, positions, base) -> np.ndarray:
+        """fp64 rotated rows of x [T, H, D] (uint16 bf16 bits) at positions [T]."""
+        T, H, D = x.shape
+        x = np.ascontiguousarray(x)
+        positions = np.ascontiguousarray(positions, dtype=np.int64)
+        out = np.zeros((T, H, D), dtype=np.float64)
+        rc = self.lib.ref_rope_rows(_ptr(out), _ptr(x), H * D, _ptr(positions), T, H, D, float(base))
+        self._check(rc, "rope_rows")
+        return out
+
+    def kv_cache_write_rope(self, key, value, k_cache, v_cache, slot_mapping, positions, base,
+                            allow_bounds=False) -> int:
+        """Cache write with K rotated at its position (bf16 of the fp64 rotation); V copied."""
+        T, Hkv, D = key.shape
+        NB, Hkv2, bs, D2 = k_cache.shape
+        assert Hkv == Hkv2 and D == D2 and value.shape == key.shape and v_cache.shape == k_cache.shape
+        slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+        positions = np.ascontiguousarray(positions, dtype=np.int64)
+        key = np.ascontiguousarray(key)
+        value = np.ascontiguousarray(value)
+        rc = self.lib.ref_kv_cache_write_rope(_ptr(key), _ptr(value), Hkv * D, Hkv * D, _ptr(k_cache),
+                                              _ptr(v_cache), _ptr(slot_mapping), _ptr(positions), T, Hkv, D, NB,
+                                              bs, float(base))
+        return self._check(rc, "kv_cache_write_rope", allow_bounds)
 
     # -- sliding window -------------------------------------------------------
     def paged_attention_window(self, q, k_cache, v_cache, block_tables, context_lens, scale, window,

@@ -714,3 +714,103 @@ int ref_paged_attention_prefill_window(double* out, const uint16_t* q,
   }
   return status;
 }
+
+/* ========================================================================= */
+/* Rotary position embedding applied to K as it is written into the cache.    */
+/*                                                                            */
+/* The fused-ops page fuses RoPE with the step before it so the rotated rows  */
+/* make one trip through memory ("Triton融合算子优化：LLM推理性能提升3倍的工  */
+/* 程实践", section 3.1); the Tiny-Infer page lists RoPE among Llama's       */
+/* operators.  Neither prints the formula.  Reading taken: Llama's form as   */
+/* the HuggingFace implementation the Tiny-Infer page checks against uses    */
+/* it: element i < D/2 pairs with i + D/2, angle pos * base^(-2i/D),          */
+/*   y[i]       = x[i] cos - x[i + D/2] sin                                  */
+/*   y[i + D/2] = x[i + D/2] cos + x[i] sin                                  */
+/* in fp64 here (exact cos/sin of the exact angle up to fp64 rounding).      */
+/* ========================================================================= */
+
+static void rope_row(double* y, const uint16_t* x, int64_t pos, int32_t D, double base) {
+  const int32_t half = D / 2;
+  for (int32_t i = 0; i < half; ++i) {
+#if PKV_ORACLE_MUTANT == 17
+    const double inv_freq = pow(base, -(double)i / (double)D); /* planted: exponent halved */
+#else
+    const double inv_freq = pow(base, -2.0 * (double)i / (double)D);
+#endif
+    const double a = (double)pos * inv_freq;
+    const double c = cos(a);
+#if PKV_ORACLE_MUTANT == 16
+    const double s = -sin(a); /* planted: rotation the other way */
+#else
+    const double s = sin(a);
+#endif
+#if PKV_ORACLE_MUTANT == 15
+    const int32_t i1 = 2 * i, i2 = 2 * i + 1; /* planted: adjacent pairs */
+#else
+    const int32_t i1 = i, i2 = i + half;
+#endif
+    const double x1 = bf16_bits_to_f64(x[i1]), x2 = bf16_bits_to_f64(x[i2]);
+    y[i1] = x1 * c - x2 * s;
+    y[i2] = x2 * c + x1 * s;
+  }
+}
+
+/* Rotated rows in fp64: x [T][H][D] bf16 bits (token stride in elements),
+ * positions [T]; out [T][H][D].  D even. */
+int ref_rope_rows(double* out, const uint16_t* x, int64_t x_stride_tok, const int64_t* positions,
+                  int64_t T, int32_t H, int32_t D, double base) {
+  if (T < 0 || H <= 0 || D <= 0 || D % 2 != 0 || !(base > 0.0)) return ORC_INVALID;
+  for (int64_t t = 0; t < T; ++t)
+    for (int32_t h = 0; h < H; ++h)
+      rope_row(out + (t * H + h) * D, x + t * x_stride_tok + (int64_t)h * D, positions[t], D, base);
+  return ORC_OK;
+}
+
+/* fp64 -> bf16 bits, round to nearest even on the value itself (no double
+ * rounding through fp32): 8 significant bits for normal values. */
+static uint16_t f64_to_bf16_bits(double v) {
+  float f;
+  if (v == 0.0 || !isfinite(v)) {
+    f = (float)v;
+  } else {
+    int e;
+    const double m = frexp(v, &e);              /* v = m * 2^e, 0.5 <= |m| < 1 */
+    const double r = nearbyint(ldexp(m, 8));    /* 8 significant bits, ties to even */
+    f = (float)ldexp(r, e - 8);                 /* exact in fp32 */
+  }
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  return (uint16_t)(u >> 16);
+}
+
+/* Cache write with K rotated at its position: K rows become bf16(rope(K)),
+ * V rows are copied; slots < 0 are skipped. */
+int ref_kv_cache_write_rope(const uint16_t* key, const uint16_t* value,
+                            int64_t key_stride_tok, int64_t value_stride_tok,
+                            uint16_t* k_cache, uint16_t* v_cache,
+                            const int64_t* slot_mapping, const int64_t* positions,
+                            int32_t T, int32_t Hkv, int32_t D, int32_t NB, int32_t bs,
+                            double base) {
+  if (T < 0 || Hkv <= 0 || D <= 0 || D % 2 != 0 || NB < 0 || bs <= 0 || !(base > 0.0))
+    return ORC_INVALID;
+  const int64_t pool_slots = (int64_t)NB * bs;
+  int status = ORC_OK;
+  double* y = (double*)malloc(sizeof(double) * D);
+  for (int64_t t = 0; t < T; ++t) {
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) continue;
+    if (slot >= pool_slots) {
+      status = ORC_BOUNDS;
+      continue;
+    }
+    const int64_t blk = slot / bs, off = slot % bs;
+    for (int32_t h = 0; h < Hkv; ++h) {
+      const int64_t dst = ((blk * Hkv + h) * bs + off) * (int64_t)D;
+      rope_row(y, key + t * key_stride_tok + (int64_t)h * D, positions[t], D, base);
+      for (int32_t d = 0; d < D; ++d) k_cache[dst + d] = f64_to_bf16_bits(y[d]);
+      memcpy(v_cache + dst, value + t * value_stride_tok + (int64_t)h * D, (size_t)D * sizeof(uint16_t));
+    }
+  }
+  free(y);
+  return status;
+}

@@ -33,7 +33,14 @@ section "分页KV缓存：借鉴操作系统的内存管理"; exact softmax atte
   inference-lab page's sliding-window cache): W >= L is full attention bit for
   bit, W = 1 returns the last key's V row, decode equals full attention over a
   contiguous cache holding only the last W keys, the last query of a prefill
-  chunk equals windowed decode, and NumPy brute force with a banded mask agrees.
+  chunk equals windowed decode, and NumPy brute force with a banded mask agrees;
+* RoPE written with K (the fused-ops page's fusion of RoPE into the step
+  before; Llama's form, element i paired with i + D/2, angle pos*base^(-2i/D)):
+  position 0 is the identity; a unit vector at D = 4 gives cos/sin of the
+  expected angles in the expected slots (pairing, sign and both frequencies);
+  pair norms are kept; dot products depend only on the position difference;
+  the cache write stores bf16 of the fp64 rotation, copies V bit for bit and
+  leaves every other slot alone.
 """
 from __future__ import annotations
 
@@ -544,6 +551,78 @@ def pin_window_prefill_brute_force_and_last_row(orc):
             assert np.array_equal(got[qsl[b + 1] - 1], last[0])
 
 
+# --------------------------------------------------------------------------- #
+# RoPE in the cache write                                                      #
+# --------------------------------------------------------------------------- #
+
+def pin_rope_position_zero_is_identity(orc):
+    rng = np.random.default_rng(51)
+    x = rand_bits(rng, (5, 3, 16))
+    y = orc.rope_rows(x, np.zeros(5, np.int64), 10000.0)
+    assert np.array_equal(y, bf16_bits_to_f64(x))
+
+
+def pin_rope_unit_vectors_d4(orc):
+    """D = 4, base 100: pair (0, 2) turns at pos * 1, pair (1, 3) at pos * 0.1."""
+    for pos in (1, 7, 123):
+        e0 = np.zeros((1, 1, 4), np.uint16)
+        e0[0, 0, 0] = 0x3F80                          # 1.0
+        y = orc.rope_rows(e0, np.array([pos]), 100.0)[0, 0]
+        assert np.allclose(y, [np.cos(pos), 0.0, np.sin(pos), 0.0], rtol=0, atol=1e-15), y
+        e1 = np.zeros((1, 1, 4), np.uint16)
+        e1[0, 0, 1] = 0x3F80
+        y = orc.rope_rows(e1, np.array([pos]), 100.0)[0, 0]
+        assert np.allclose(y, [0.0, np.cos(0.1 * pos), 0.0, np.sin(0.1 * pos)], rtol=0, atol=1e-15), y
+
+
+def pin_rope_keeps_norms_and_relative_position(orc):
+    rng = np.random.default_rng(52)
+    D = 32
+    q = rand_bits(rng, (1, 1, D))
+    k = rand_bits(rng, (1, 1, D))
+    x = bf16_bits_to_f64(q)[0, 0]
+    y = orc.rope_rows(q, np.array([4321]), 500000.0)[0, 0]
+    h = D // 2
+    assert np.allclose(y[:h] ** 2 + y[h:] ** 2, x[:h] ** 2 + x[h:] ** 2, rtol=1e-13, atol=0)
+    for m, n, sft in ((5, 2, 100), (1000, 17, 3), (0, 99, 12345)):
+        a = np.dot(orc.rope_rows(q, np.array([m]), 10000.0)[0, 0], orc.rope_rows(k, np.array([n]), 10000.0)[0, 0])
+        b = np.dot(orc.rope_rows(q, np.array([m + sft]), 10000.0)[0, 0],
+                   orc.rope_rows(k, np.array([n + sft]), 10000.0)[0, 0])
+        assert abs(a - b) <= 1e-11 * max(1.0, abs(a)), (a, b)
+
+
+def pin_rope_cache_write(orc):
+    rng = np.random.default_rng(53)
+    T, Hkv, D, bs, NB = 9, 2, 16, 4, 5
+    key = rand_bits(rng, (T, Hkv, D))
+    val = rand_bits(rng, (T, Hkv, D))
+    k = rand_bits(rng, (NB, Hkv, bs, D))
+    v = rand_bits(rng, (NB, Hkv, bs, D))
+    k0, v0 = k.copy(), v.copy()
+    slots = np.array([3, -1, 0, 19, 7, 8, -1, 12, 1], np.int64)
+    pos = rng.integers(0, 100000, size=T).astype(np.int64)
+    orc.kv_cache_write_rope(key, val, k, v, slots, pos, 500000.0)
+    want = orc.rope_rows(key, pos, 500000.0)
+    for t, sl in enumerate(slots):
+        if sl < 0:
+            continue
+        blk, off = sl // bs, sl % bs
+        got = bf16_bits_to_f64(k[blk, :, off])
+        # bf16 of the fp64 value: within half a bf16 step, 8 significant bits,
+        # i.e. at most 2^-8 relative (at the bottom of a binade)
+        assert np.all(np.abs(got - want[t]) <= np.abs(want[t]) * 2.0 ** -8 + 1e-300)
+        # and it is the nearest bf16: the neighbours one step away are farther
+        bits = k[blk, :, off].astype(np.int64)
+        for nb in (bits - 1, bits + 1):
+            other = bf16_bits_to_f64(nb.astype(np.uint16))
+            ok = np.isnan(other) | (np.abs(other - want[t]) >= np.abs(got - want[t]))
+            assert np.all(ok)
+        assert np.array_equal(v[blk, :, off], val[t])
+        k0[blk, :, off] = k[blk, :, off]
+        v0[blk, :, off] = v[blk, :, off]
+    assert np.array_equal(k, k0) and np.array_equal(v, v0)   # nothing else touched
+
+
 ALL_PINS = [
     pin_golden_closed_form,
     pin_brute_force_decode,
@@ -568,4 +647,8 @@ ALL_PINS = [
     pin_window_one_returns_last_v,
     pin_window_equals_truncated_context,
     pin_window_prefill_brute_force_and_last_row,
+    pin_rope_position_zero_is_identity,
+    pin_rope_unit_vectors_d4,
+    pin_rope_keeps_norms_and_relative_position,
+    pin_rope_cache_write,
 ]
