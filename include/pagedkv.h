@@ -119,6 +119,29 @@ size_t pkv_paged_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv,
                                           int32_t max_context_len_hint);
 
 /*
+ * kv_cache_write_rope -- pkv_kv_cache_write with rotary position embedding
+ * applied to K on the way in, so the rotated rows make one trip through
+ * memory (the fused-ops page fuses RoPE into the step before it:
+ * "Triton融合算子优化：LLM推理性能提升3倍的工程实践", section 3.1).  The pages
+ * print no formula; Llama's form (as in the HuggingFace implementation the
+ * Tiny-Infer page checks against) is used: element i < D/2 pairs with
+ * i + D/2 and turns by pos * rope_base^(-2i/D),
+ *   k'[i] = k[i] cos - k[i+D/2] sin,  k'[i+D/2] = k[i+D/2] cos + k[i] sin.
+ * The angle is formed and reduced in fp64, sine/cosine and the rotation in
+ * fp32, one bf16 rounding at the end.  V rows are copied bit for bit.
+ *   positions : device, [T] int64, the absolute position of each token
+ *   rope_base : > 1 (10000 for Llama 2, 500000 for Llama 3)
+ * Other arguments and errors as pkv_kv_cache_write (D even, 2-byte aligned).
+ */
+pkv_status pkv_kv_cache_write_rope(const void* key, const void* value,
+                                   int64_t key_stride_tok,
+                                   int64_t value_stride_tok, void* k_cache,
+                                   void* v_cache, const int64_t* slot_mapping,
+                                   const int64_t* positions, int32_t T, int32_t Hkv,
+                                   int32_t D, int32_t NB, int32_t bs, double rope_base,
+                                   pkv_dtype dtype, pkv_stream_t stream);
+
+/*
  * INT8 KV cache.  The Tiny-Infer page (section "推测性解码与INT8量化") names
  * an INT8 KV cache as the way to halve its memory; it fixes neither the scale
  * granularity nor the rounding.  This library's reading: symmetric codes with

@@ -13,6 +13,7 @@ Calls (same names as the C ABI):
     paged_attention_split(..., pages_per_split)
     paged_attention_prefill(q, query_start_loc, k_cache, v_cache, block_tables,
                             context_lens, scale, max_q_len, ...)
+    kv_cache_write_rope(key, value, k_cache, v_cache, slot_mapping, positions, rope_base)
     kv_cache_write_int8(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping)
     paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables,
                          context_lens, scale, ...)
@@ -54,6 +55,8 @@ EXPORTS = {
     "pkv_split_workspace_size": ([_I32, _I32, _I32, _I32], _SZ),
     "pkv_paged_attention_split_noalloc": ([_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                            _I32, _F32, _I32, _I32, _I32, _P], _I32),
+    "pkv_kv_cache_write_rope": ([_P, _P, _I64, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32,
+                                 ctypes.c_double, _I32, _P], _I32),
     "pkv_kv_cache_write_int8": ([_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
     "pkv_paged_attention_int8": ([_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32,
                                   _I32, _P, _SZ, _P], _I32),
@@ -170,6 +173,27 @@ def _decode_common(q, k_cache, v_cache, block_tables, context_lens, out):
         if out.shape != q.shape:
             raise ValueError("out must have q's shape")
     return NB, Hkv, bs, D, B, Hq, block_tables.shape[1], out
+
+
+def kv_cache_write_rope(key, value, k_cache, v_cache, slot_mapping, positions, rope_base: float,
+                        stream=None) -> None:
+    """Cache write with K rotated by RoPE at ``positions`` [T] (int64) on the way in."""
+    for t, name in ((key, "key"), (value, "value")):
+        _dev(t, name, torch.bfloat16)
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be [T, Hkv, D] with contiguous (head, dim)")
+    NB, Hkv, bs, D = _cache_dims(k_cache, v_cache)
+    _contig(_dev(slot_mapping, "slot_mapping", torch.int64), "slot_mapping")
+    _contig(_dev(positions, "positions", torch.int64), "positions")
+    T = key.shape[0]
+    if key.shape[1:] != (Hkv, D) or value.shape != key.shape or slot_mapping.numel() != T \
+            or positions.numel() != T:
+        raise ValueError("shape mismatch between key/value, caches, slot_mapping and positions")
+    rc = load_library().pkv_kv_cache_write_rope(
+        key.data_ptr(), value.data_ptr(), key.stride(0), value.stride(0), k_cache.data_ptr(), v_cache.data_ptr(),
+        slot_mapping.data_ptr(), positions.data_ptr(), T, Hkv, D, NB, bs, float(rope_base), PKV_BF16,
+        _stream(stream))
+    _check(rc, "kv_cache_write_rope")
 
 
 def kv_cache_write_int8(key, value, k_cache, v_cache, k_scale, v_scale, slot_mapping, stream=None) -> None:

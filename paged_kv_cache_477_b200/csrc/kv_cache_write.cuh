@@ -127,3 +127,64 @@ __global__ void __launch_bounds__(256) kv_cache_write_i8_kernel(const __grid_con
 }
 
 }  // namespace pkv
+
+namespace pkv {
+
+// ---------------------------------------------------------------------------
+// Cache write with RoPE applied to K on the way in, so the rotated rows make
+// one trip through memory (the fused-ops page fuses RoPE into the step before
+// it, section 3.1).  The pages print no formula; Llama's form is used, as in
+// the HuggingFace implementation the Tiny-Infer page checks against: element i
+// < D/2 pairs with i + D/2 and turns by pos * base^(-2i/D):
+//   k'[i] = k[i] cos - k[i + D/2] sin,   k'[i + D/2] = k[i + D/2] cos + k[i] sin.
+// The angle is formed and reduced to [-pi, pi] in fp64 (an fp32 product of
+// position and frequency would be off by ~1e-3 rad at 10^5 positions), then
+// sine and cosine are taken in fp32 and the rotation is rounded once to bf16.
+// V rows are copied.  One thread per (token, kv head, pair).
+// ---------------------------------------------------------------------------
+struct KvWriteRopeParams {
+  const __nv_bfloat16* key;   // [T][Hkv][D], token stride given
+  const __nv_bfloat16* value;
+  int64_t key_stride, value_stride;  // elements
+  __nv_bfloat16* k_cache;     // [NB][Hkv][bs][D]
+  __nv_bfloat16* v_cache;
+  const int64_t* slot_mapping;
+  const int64_t* positions;   // [T]
+  int64_t total;              // T * Hkv * D/2
+  int64_t pool_slots;
+  int32_t Hkv, D, bs;
+  double log2_base;           // log2(rope base)
+};
+
+__global__ void __launch_bounds__(256) kv_cache_write_rope_kernel(const __grid_constant__ KvWriteRopeParams p) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= p.total) return;
+  const int half = p.D / 2;
+  const int i = (int)(idx % half);
+  const int64_t th = idx / half;
+  const int h = (int)(th % p.Hkv);
+  const int64_t t = th / p.Hkv;
+  const int64_t slot = __ldg(p.slot_mapping + t);
+  if (slot < 0) return;  // padding token
+  if (slot >= p.pool_slots) {
+    if (i == 0) set_error(PKV_ERR_BOUNDS);
+    return;
+  }
+  const int64_t pos = __ldg(p.positions + t);
+  const double inv_freq = exp2(-2.0 * (double)i / (double)p.D * p.log2_base);
+  const double a = (double)pos * inv_freq;
+  const double two_pi = 6.283185307179586;
+  const float r = (float)(a - two_pi * rint(a / two_pi));  // in [-pi, pi]
+  float sn, cs;
+  sincosf(r, &sn, &cs);
+  const __nv_bfloat16* kr = p.key + t * p.key_stride + (int64_t)h * p.D;
+  const __nv_bfloat16* vr = p.value + t * p.value_stride + (int64_t)h * p.D;
+  const float x1 = __bfloat162float(kr[i]), x2 = __bfloat162float(kr[i + half]);
+  const int64_t dst = ((slot / p.bs * p.Hkv + h) * p.bs + slot % p.bs) * p.D;
+  p.k_cache[dst + i] = __float2bfloat16_rn(fmaf(x1, cs, -x2 * sn));
+  p.k_cache[dst + i + half] = __float2bfloat16_rn(fmaf(x2, cs, x1 * sn));
+  p.v_cache[dst + i] = vr[i];
+  p.v_cache[dst + i + half] = vr[i + half];
+}
+
+}  // namespace pkv

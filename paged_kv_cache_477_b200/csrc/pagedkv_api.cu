@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -468,6 +469,43 @@ size_t pkv_paged_attention_window_workspace_size(int32_t B, int32_t Hq, int32_t 
     return 0;
   const int32_t span = (int32_t)std::min<int64_t>((int64_t)window_pages(window) * bs, (int64_t)MB * bs);
   return plan_auto(B, Hq, Hkv, D, MB, bs, span).workspace;
+}
+
+pkv_status pkv_kv_cache_write_rope(const void* key, const void* value, int64_t key_stride_tok,
+                                   int64_t value_stride_tok, void* k_cache, void* v_cache,
+                                   const int64_t* slot_mapping, const int64_t* positions, int32_t T,
+                                   int32_t Hkv, int32_t D, int32_t NB, int32_t bs, double rope_base,
+                                   pkv_dtype dtype, pkv_stream_t stream) {
+  t_launches = 0;
+  if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (T < 0 || Hkv <= 0 || D <= 0 || D % 2 != 0 || NB < 0 || bs <= 0 || !(rope_base > 1.0) ||
+      !std::isfinite(rope_base))
+    return PKV_ERR_INVALID_ARG;
+  if (T == 0) return PKV_OK;
+  if (!key || !value || !k_cache || !v_cache || !slot_mapping || !positions) return PKV_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(key) | reinterpret_cast<uintptr_t>(value) |
+        reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 1) != 0)
+    return PKV_ERR_INVALID_ARG;
+  if (key_stride_tok < (int64_t)Hkv * D || value_stride_tok < (int64_t)Hkv * D) return PKV_ERR_INVALID_ARG;
+  pkv::KvWriteRopeParams p{};
+  p.key = static_cast<const __nv_bfloat16*>(key);
+  p.value = static_cast<const __nv_bfloat16*>(value);
+  p.key_stride = key_stride_tok;
+  p.value_stride = value_stride_tok;
+  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p.slot_mapping = slot_mapping;
+  p.positions = positions;
+  p.total = (int64_t)T * Hkv * (D / 2);
+  p.pool_slots = (int64_t)NB * bs;
+  p.Hkv = Hkv; p.D = D; p.bs = bs;
+  p.log2_base = std::log2(rope_base);
+  const int64_t blocks = (p.total + 255) / 256;
+  if (blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
+  pkv::kv_cache_write_rope_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  pkv_status s = launch_status();
+  if (s == PKV_OK) t_launches = 1;
+  return s;
 }
 
 size_t pkv_split_workspace_size(int32_t B, int32_t Hq, int32_t D, int32_t num_splits) {

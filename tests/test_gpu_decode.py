@@ -12,6 +12,7 @@ import oracle
 import paged_kv_cache_477_b200 as pkv
 from paged_kv_cache_477_b200 import workloads as wl
 from paged_kv_cache_477_b200.workloads import bf16_bits
+from oracle import bf16_bits_to_f64
 from parity import HostCase, assert_close
 
 pytestmark = pytest.mark.gpu
@@ -272,3 +273,62 @@ def test_decode_window_rejects_zero():
     with pytest.raises(pkv.PagedKVError):
         pkv.paged_attention_window(case.q, case.k_cache, case.v_cache, case.block_tables,
                                    case.context_lens, case.scale, 0)
+
+
+# --------------------------------------------------------------------------- #
+# RoPE fused into the cache write                                              #
+# --------------------------------------------------------------------------- #
+
+@pytest.mark.parametrize("T,Hkv,D,bs,NB,base", [(37, 2, 64, 16, 9, 10000.0), (128, 8, 128, 16, 64, 500000.0),
+                                               (6, 3, 256, 4, 4, 10000.0)])
+def test_kv_cache_write_rope(T, Hkv, D, bs, NB, base):
+    """Rotated K rows within half a bf16 step of the fp64 rotation (plus fp32
+    slack on the pair); V rows and every untouched slot bit-exact."""
+    g = torch.Generator(device="cuda").manual_seed(T * 3 + D)
+    k_cache = torch.randn(NB, Hkv, bs, D, device="cuda", generator=g).to(torch.bfloat16)
+    v_cache = torch.randn(NB, Hkv, bs, D, device="cuda", generator=g).to(torch.bfloat16)
+    key = torch.randn(T, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
+    val = torch.randn(T, Hkv, D, device="cuda", generator=g).to(torch.bfloat16)
+    gc = torch.Generator().manual_seed(T)
+    slots = torch.randperm(NB * bs, generator=gc)[:T].to(torch.int64)
+    slots[::5] = -1
+    pos = torch.randint(0, 131072, (T,), generator=gc, dtype=torch.int64)
+    pos[0] = 0
+    k_before, v_before = bf16_bits(k_cache).copy(), bf16_bits(v_cache).copy()
+    pkv.kv_cache_write_rope(key, val, k_cache, v_cache, slots.cuda(), pos.cuda(), base)
+    assert pkv.last_launch_count() == 1
+    want = oracle.get().rope_rows(bf16_bits(key), pos.numpy(), base)       # fp64 [T, Hkv, D]
+    kb, vb = bf16_bits(k_cache), bf16_bits(v_cache)
+    x = np.abs(bf16_bits_to_f64(bf16_bits(key)))
+    half = D // 2
+    pair = x[..., :half] + x[..., half:]
+    pair = np.concatenate([pair, pair], axis=-1)
+    for t, sl in enumerate(slots.tolist()):
+        if sl < 0:
+            continue
+        blk, off = sl // bs, sl % bs
+        got = bf16_bits_to_f64(kb[blk, :, off])
+        bound = np.abs(want[t]) * 2.0 ** -8 + pair[t] * 2.0 ** -20
+        assert np.all(np.abs(got - want[t]) <= bound), (t, np.abs(got - want[t]).max())
+        assert np.array_equal(vb[blk, :, off], bf16_bits(val)[t])
+        k_before[blk, :, off] = kb[blk, :, off]
+        v_before[blk, :, off] = vb[blk, :, off]
+    assert np.array_equal(kb, k_before) and np.array_equal(vb, v_before)
+    _no_device_error()
+
+
+def test_rope_write_then_decode():
+    """Decode over a cache whose newest rows were rotated on the way in,
+    against the oracle's own rotated write (nothing taken from the GPU)."""
+    case = wl.workload("llama3_8b_decode", device="cuda", B=16, lens=[4096] * 16)
+    host = HostCase(case)
+    pos = (case.context_lens.to(torch.int64) - 1)                       # the new token's position
+    pkv.kv_cache_write_rope(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping, pos,
+                            500000.0)
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale, max_context_len=4096)
+    oracle.get().kv_cache_write_rope(bf16_bits(case.new_key), bf16_bits(case.new_value), host.k, host.v,
+                                     case.slot_mapping.cpu().numpy(), pos.cpu().numpy(), 500000.0)
+    host.written = True
+    assert_close(out, host.decode_ref(), "rope write + decode")
+    _no_device_error()
