@@ -56,7 +56,8 @@ typedef enum pkv_status {
   PKV_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed            */
   PKV_ERR_TIMEOUT = 4,      /* device: a bounded wait gave up                  */
   PKV_ERR_BOUNDS = 5,       /* device: slot / block id / length out of range   */
-  PKV_ERR_WORKSPACE = 6     /* workspace missing or smaller than required      */
+  PKV_ERR_WORKSPACE = 6,    /* workspace missing or smaller than required      */
+  PKV_ERR_NO_BLOCKS = 7     /* block allocator: not enough free blocks         */
 } pkv_status;
 
 typedef enum pkv_dtype { PKV_BF16 = 0 } pkv_dtype;
@@ -304,6 +305,57 @@ pkv_status pkv_paged_attention_prefill_window(
     int32_t MB, const int32_t* context_lens, int32_t B, int32_t sumQ,
     int32_t max_q_len, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
     int32_t bs, float scale, int32_t window, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * Shared blocks and copy-on-write.  Sequences that share a prefix (parallel
+ * sampling from one prompt) can point their block tables at the same
+ * physical blocks and copy a block only when one of them is about to write
+ * into it -- the vLLM-style block copying the Tiny-Infer page plans for its
+ * paged cache (section "分页KV缓存：借鉴操作系统的内存管理").
+ *
+ * pkv_block_allocator_*: host-only bookkeeping of which physical blocks are
+ * in use and by how many holders (no device memory, no CUDA calls; one mutex
+ * per allocator, so host threads may share one).  A fresh allocator hands out
+ * the lowest ids first.  Every call is all-or-nothing: on an error nothing
+ * changes.
+ *   create(num_blocks, &a)          num_blocks >= 0; destroy(a) frees it.
+ *   alloc(a, n, ids)                n fresh blocks, refcount 1, written to ids
+ *                                   (host array of n); PKV_ERR_NO_BLOCKS if
+ *                                   fewer than n are free.
+ *   share(a, ids, n)                refcount + 1 for each (all must be live).
+ *   release(a, ids, n)              refcount - 1 for each; blocks reaching 0
+ *                                   are free again (ids may repeat).
+ *   cow(a, id, &new_id, &copy)      before writing into block id: if it is
+ *                                   shared, new_id is a fresh block for the
+ *                                   writer, id loses one holder, copy = 1 and
+ *                                   the caller must pkv_copy_blocks(id ->
+ *                                   new_id) before writing; if private,
+ *                                   new_id = id and copy = 0.
+ *   num_free(a), refcount(a, id)    queries (refcount -1: id outside the pool).
+ */
+typedef struct pkv_block_allocator pkv_block_allocator;
+pkv_status pkv_block_allocator_create(int32_t num_blocks, pkv_block_allocator** out);
+void pkv_block_allocator_destroy(pkv_block_allocator* a);
+pkv_status pkv_block_allocator_alloc(pkv_block_allocator* a, int32_t n, int32_t* ids);
+pkv_status pkv_block_allocator_share(pkv_block_allocator* a, const int32_t* ids, int32_t n);
+pkv_status pkv_block_allocator_release(pkv_block_allocator* a, const int32_t* ids, int32_t n);
+pkv_status pkv_block_allocator_cow(pkv_block_allocator* a, int32_t id, int32_t* new_id,
+                                   int32_t* must_copy);
+int32_t pkv_block_allocator_num_free(pkv_block_allocator* a);
+int32_t pkv_block_allocator_refcount(pkv_block_allocator* a, int32_t id);
+
+/*
+ * copy_blocks -- for each (src, dst) pair in `pairs` (device, [n][2] int32)
+ * copy block src to block dst, bit for bit, in both pools (k_cache and
+ * v_cache; for the INT8 cache call once for the codes and once for the
+ * scales).  block_bytes: bytes of one block of one pool (Hkv*bs*D*elem),
+ * a multiple of 16; pools 16-byte aligned.  A dst must not also be a src in
+ * the same call, nor appear twice (the pairs run concurrently).  A block id outside [0, NB) sets PKV_ERR_BOUNDS on the
+ * device and that pair is skipped.  One launch (none if n = 0).
+ */
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, size_t block_bytes,
+                           const int32_t* pairs, int32_t n, int32_t NB,
+                           pkv_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads and clears the current device's error

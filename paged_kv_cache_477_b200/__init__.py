@@ -20,6 +20,7 @@ Calls (same names as the C ABI):
     paged_attention_window(q, k_cache, v_cache, block_tables, context_lens, scale, window, ...)
     paged_attention_prefill_window(q, query_start_loc, k_cache, v_cache, block_tables,
                                    context_lens, scale, max_q_len, window, ...)
+    copy_blocks(k_cache, v_cache, pairs);  BlockAllocator(num_blocks)
 """
 from __future__ import annotations
 
@@ -35,7 +36,7 @@ LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
 PKV_BF16 = 0
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "CUDA error",
           4: "device wait timed out", 5: "index out of range on the device",
-          6: "workspace missing or too small"}
+          6: "workspace missing or too small", 7: "not enough free blocks"}
 
 _lib = None
 
@@ -67,6 +68,15 @@ EXPORTS = {
                                      _I32, _I32, _I32, _F32, _I32, _P], _I32),
     "pkv_paged_attention_prefill_window": ([_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                             _I32, _I32, _I32, _F32, _I32, _I32, _P], _I32),
+    "pkv_block_allocator_create": ([_I32, ctypes.POINTER(_P)], _I32),
+    "pkv_block_allocator_destroy": ([_P], None),
+    "pkv_block_allocator_alloc": ([_P, _I32, _P], _I32),
+    "pkv_block_allocator_share": ([_P, _P, _I32], _I32),
+    "pkv_block_allocator_release": ([_P, _P, _I32], _I32),
+    "pkv_block_allocator_cow": ([_P, _I32, ctypes.POINTER(_I32), ctypes.POINTER(_I32)], _I32),
+    "pkv_block_allocator_num_free": ([_P], _I32),
+    "pkv_block_allocator_refcount": ([_P, _I32], _I32),
+    "pkv_copy_blocks": ([_P, _P, _SZ, _P, _I32, _I32, _P], _I32),
     "pkv_get_device_error": ([_P, ctypes.POINTER(_I32)], _I32),
     "pkv_last_launch_count": ([], _I32),
     "pkv_status_string": ([_I32], ctypes.c_char_p),
@@ -398,6 +408,74 @@ def paged_attention_prefill_window(q, query_start_loc, k_cache, v_cache, block_t
         B, sumQ, int(max_q_len), Hq, Hkv, D, NB, bs, float(scale), int(window), PKV_BF16, _stream(stream))
     _check(rc, "paged_attention_prefill_window")
     return out
+
+
+class BlockAllocator:
+    """Host bookkeeping of physical cache blocks with reference counts (the
+    library's pkv_block_allocator_*; no device memory, no CUDA calls)."""
+
+    def __init__(self, num_blocks: int):
+        self._lib = load_library()
+        h = _P()
+        _check(self._lib.pkv_block_allocator_create(int(num_blocks), ctypes.byref(h)), "block_allocator_create")
+        self._h = h
+
+    def close(self):
+        if self._h:
+            self._lib.pkv_block_allocator_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @staticmethod
+    def _ids(ids):
+        arr = (_I32 * len(ids))(*[int(i) for i in ids])
+        return arr, len(ids)
+
+    def alloc(self, n: int) -> list:
+        arr = (_I32 * max(1, n))()
+        _check(self._lib.pkv_block_allocator_alloc(self._h, int(n), arr), "block_allocator_alloc")
+        return list(arr[:n])
+
+    def share(self, ids) -> None:
+        arr, n = self._ids(ids)
+        _check(self._lib.pkv_block_allocator_share(self._h, arr, n), "block_allocator_share")
+
+    def release(self, ids) -> None:
+        arr, n = self._ids(ids)
+        _check(self._lib.pkv_block_allocator_release(self._h, arr, n), "block_allocator_release")
+
+    def cow(self, block: int):
+        """(block to write into, whether the caller must copy the old block to it first)."""
+        nid, must = _I32(0), _I32(0)
+        _check(self._lib.pkv_block_allocator_cow(self._h, int(block), ctypes.byref(nid), ctypes.byref(must)),
+               "block_allocator_cow")
+        return int(nid.value), bool(must.value)
+
+    def num_free(self) -> int:
+        return int(self._lib.pkv_block_allocator_num_free(self._h))
+
+    def refcount(self, block: int) -> int:
+        return int(self._lib.pkv_block_allocator_refcount(self._h, int(block)))
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, pairs: torch.Tensor, stream=None) -> None:
+    """Copy block pairs[i, 0] -> pairs[i, 1] in both pools, bit for bit.
+    Pools [NB, ...] (any dtype, contiguous); pairs int32 [n, 2] on the device."""
+    for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _contig(_dev(t, name), name)
+    _contig(_dev(pairs, "pairs", torch.int32), "pairs")
+    if k_cache.shape[0] != v_cache.shape[0] or k_cache[0].nbytes != v_cache[0].nbytes:
+        raise ValueError("k_cache and v_cache must have the same number and size of blocks")
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [n, 2]")
+    rc = load_library().pkv_copy_blocks(k_cache.data_ptr(), v_cache.data_ptr(), k_cache[0].nbytes,
+                                        pairs.data_ptr(), pairs.shape[0], k_cache.shape[0], _stream(stream))
+    _check(rc, "copy_blocks")
 
 
 def get_device_error(stream=None) -> int:

@@ -188,3 +188,33 @@ __global__ void __launch_bounds__(256) kv_cache_write_rope_kernel(const __grid_c
 }
 
 }  // namespace pkv
+
+namespace pkv {
+
+// ---------------------------------------------------------------------------
+// copy_blocks: for each (src, dst) pair copy a whole physical block (every kv
+// head's page) of each of two pools, bit for bit -- the device half of
+// copy-on-write for blocks shared between sequences (Tiny-Infer page,
+// section "分页KV缓存：借鉴操作系统的内存管理").  One CTA per pair and pool,
+// 16-byte vectors, coalesced.
+// ---------------------------------------------------------------------------
+struct CopyBlocksParams {
+  uint4* pool[2];            // k and v (or codes and scales): [NB][block_vec] 16-byte vectors
+  int64_t block_vec;         // 16-byte vectors per block
+  const int32_t* pairs;      // [n][2]: src, dst
+  int32_t n, NB;
+};
+
+__global__ void __launch_bounds__(256) copy_blocks_kernel(const __grid_constant__ CopyBlocksParams p) {
+  const int pair = blockIdx.x, which = blockIdx.y;
+  const int32_t src = __ldg(p.pairs + 2 * pair), dst = __ldg(p.pairs + 2 * pair + 1);
+  if (src < 0 || src >= p.NB || dst < 0 || dst >= p.NB) {
+    if (threadIdx.x == 0) set_error(PKV_ERR_BOUNDS);
+    return;
+  }
+  const uint4* s = p.pool[which] + (int64_t)src * p.block_vec;
+  uint4* d = p.pool[which] + (int64_t)dst * p.block_vec;
+  for (int64_t i = threadIdx.x; i < p.block_vec; i += blockDim.x) d[i] = s[i];
+}
+
+}  // namespace pkv

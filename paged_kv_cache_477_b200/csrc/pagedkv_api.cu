@@ -6,12 +6,14 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <new>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
 
 #include <cuda.h>
 
+#include "block_allocator.hpp"
 #include "decode_attn.cuh"
 #include "kv_cache_write.cuh"
 #include "pkv_common.cuh"
@@ -332,6 +334,7 @@ const char* pkv_status_string(pkv_status s) {
     case PKV_ERR_TIMEOUT: return "device wait timed out";
     case PKV_ERR_BOUNDS: return "index out of range on the device";
     case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case PKV_ERR_NO_BLOCKS: return "not enough free blocks";
   }
   return "unknown status";
 }
@@ -503,6 +506,70 @@ pkv_status pkv_kv_cache_write_rope(const void* key, const void* value, int64_t k
   const int64_t blocks = (p.total + 255) / 256;
   if (blocks > INT32_MAX) return PKV_ERR_INVALID_ARG;
   pkv::kv_cache_write_rope_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  pkv_status s = launch_status();
+  if (s == PKV_OK) t_launches = 1;
+  return s;
+}
+
+// ------------------------------------------------------- shared blocks --
+struct pkv_block_allocator {
+  pkv::BlockAllocator impl;
+  explicit pkv_block_allocator(int32_t n) : impl(n) {}
+};
+
+pkv_status pkv_block_allocator_create(int32_t num_blocks, pkv_block_allocator** out) {
+  if (!out || num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  *out = new (std::nothrow) pkv_block_allocator(num_blocks);
+  return *out ? PKV_OK : PKV_ERR_INVALID_ARG;
+}
+
+void pkv_block_allocator_destroy(pkv_block_allocator* a) { delete a; }
+
+pkv_status pkv_block_allocator_alloc(pkv_block_allocator* a, int32_t n, int32_t* ids) {
+  if (!a || n < 0 || (n > 0 && !ids)) return PKV_ERR_INVALID_ARG;
+  return a->impl.alloc(n, ids) ? PKV_OK : PKV_ERR_NO_BLOCKS;
+}
+
+pkv_status pkv_block_allocator_share(pkv_block_allocator* a, const int32_t* ids, int32_t n) {
+  if (!a || n < 0 || (n > 0 && !ids)) return PKV_ERR_INVALID_ARG;
+  return a->impl.share(ids, n) ? PKV_OK : PKV_ERR_INVALID_ARG;
+}
+
+pkv_status pkv_block_allocator_release(pkv_block_allocator* a, const int32_t* ids, int32_t n) {
+  if (!a || n < 0 || (n > 0 && !ids)) return PKV_ERR_INVALID_ARG;
+  return a->impl.release(ids, n) ? PKV_OK : PKV_ERR_INVALID_ARG;
+}
+
+pkv_status pkv_block_allocator_cow(pkv_block_allocator* a, int32_t id, int32_t* new_id, int32_t* must_copy) {
+  if (!a || !new_id || !must_copy) return PKV_ERR_INVALID_ARG;
+  if (a->impl.refcount(id) <= 0) return PKV_ERR_INVALID_ARG;
+  bool copy = false;
+  int32_t nid = -1;
+  if (!a->impl.copy_on_write(id, &nid, &copy)) return PKV_ERR_NO_BLOCKS;
+  *new_id = nid;
+  *must_copy = copy ? 1 : 0;
+  return PKV_OK;
+}
+
+int32_t pkv_block_allocator_num_free(pkv_block_allocator* a) { return a ? a->impl.num_free() : -1; }
+
+int32_t pkv_block_allocator_refcount(pkv_block_allocator* a, int32_t id) { return a ? a->impl.refcount(id) : -1; }
+
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, size_t block_bytes, const int32_t* pairs, int32_t n,
+                           int32_t NB, pkv_stream_t stream) {
+  t_launches = 0;
+  if (n < 0 || NB < 0 || block_bytes == 0 || block_bytes % 16 != 0) return PKV_ERR_INVALID_ARG;
+  if (n == 0) return PKV_OK;
+  if (!k_cache || !v_cache || !pairs || !aligned16(k_cache) || !aligned16(v_cache)) return PKV_ERR_INVALID_ARG;
+  if (n > 65535 * 64) return PKV_ERR_UNSUPPORTED;
+  pkv::CopyBlocksParams p{};
+  p.pool[0] = static_cast<uint4*>(k_cache);
+  p.pool[1] = static_cast<uint4*>(v_cache);
+  p.block_vec = (int64_t)(block_bytes / 16);
+  p.pairs = pairs;
+  p.n = n;
+  p.NB = NB;
+  pkv::copy_blocks_kernel<<<dim3(n, 2), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
   pkv_status s = launch_status();
   if (s == PKV_OK) t_launches = 1;
   return s;
