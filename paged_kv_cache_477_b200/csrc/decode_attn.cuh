@@ -227,47 +227,15 @@ __device__ __forceinline__ void widen_i8x4(uint32_t w, float2& lo, float2& hi) {
                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7543))), bias);
 }
 
-template <int D, int HG, int ROWS>
-__device__ __forceinline__ void attend_rows_i8(LaneState<HG>& st, const float2 (&q2)[HG][8],
-                                               const unsigned char* kp, const unsigned char* vp,
-                                               const float* ksc, const float* vsc, int nstart, int nvalid,
-                                               int rg, int sub) {
-  constexpr int LPR = D / 16, RPW = 32 / LPR, TPL = ROWS / RPW;
-  float sc[TPL][HG];
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    const int r = rg + t * RPW;
-    const uint4 ka = reinterpret_cast<const uint4*>(kp + r * D)[sub];
-    float2 k2[8];
-    widen_i8x4(ka.x, k2[0], k2[1]);
-    widen_i8x4(ka.y, k2[2], k2[3]);
-    widen_i8x4(ka.z, k2[4], k2[5]);
-    widen_i8x4(ka.w, k2[6], k2[7]);
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      float2 d = __fmul2_rn(q2[h][0], k2[0]);
-#pragma unroll
-      for (int e = 1; e < 8; ++e) d = __ffma2_rn(q2[h][e], k2[e], d);
-      sc[t][h] = d.x + d.y;
-    }
-  }
-#pragma unroll
-  for (int off = LPR / 2; off >= 1; off >>= 1)
-#pragma unroll
-    for (int t = 0; t < TPL; ++t)
-#pragma unroll
-      for (int h = 0; h < HG; ++h) sc[t][h] += __shfl_xor_sync(0xffffffffu, sc[t][h], off);
-
-  bool valid[TPL];
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    const int r = rg + t * RPW;
-    valid[t] = r < nvalid && r >= nstart;
-    const float ks = valid[t] ? ksc[r] : 0.f;  // rows outside the range are never read
-#pragma unroll
-    for (int h = 0; h < HG; ++h) sc[t][h] *= ks;
-  }
-
+// Online softmax and P.V over TPL rows of int8 V codes (row stride D bytes,
+// one fp32 scale per row in vsc): sc[t][h] are the rows' scores (log2
+// domain), valid[t] whether row rg + t * RPW takes part.  Invalid rows take no
+// part in the max and are never read from V.
+template <int D, int HG, int TPL>
+__device__ __forceinline__ void softmax_pv_i8(LaneState<HG>& st, const float (&sc)[TPL][HG],
+                                              const bool (&valid)[TPL], const unsigned char* vp,
+                                              const float* vsc, int rg, int sub) {
+  constexpr int RPW = 32 / (D / 16);
   float mp[HG];
   bool grow = false;
 #pragma unroll
@@ -311,6 +279,49 @@ __device__ __forceinline__ void attend_rows_i8(LaneState<HG>& st, const float2 (
       for (int e = 0; e < 8; ++e) st.acc[h][e] = __ffma2_rn(pp, v2[e], st.acc[h][e]);
     }
   }
+}
+
+template <int D, int HG, int ROWS>
+__device__ __forceinline__ void attend_rows_i8(LaneState<HG>& st, const float2 (&q2)[HG][8],
+                                               const unsigned char* kp, const unsigned char* vp,
+                                               const float* ksc, const float* vsc, int nstart, int nvalid,
+                                               int rg, int sub) {
+  constexpr int LPR = D / 16, RPW = 32 / LPR, TPL = ROWS / RPW;
+  float sc[TPL][HG];
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) {
+    const int r = rg + t * RPW;
+    const uint4 ka = reinterpret_cast<const uint4*>(kp + r * D)[sub];
+    float2 k2[8];
+    widen_i8x4(ka.x, k2[0], k2[1]);
+    widen_i8x4(ka.y, k2[2], k2[3]);
+    widen_i8x4(ka.z, k2[4], k2[5]);
+    widen_i8x4(ka.w, k2[6], k2[7]);
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      float2 d = __fmul2_rn(q2[h][0], k2[0]);
+#pragma unroll
+      for (int e = 1; e < 8; ++e) d = __ffma2_rn(q2[h][e], k2[e], d);
+      sc[t][h] = d.x + d.y;
+    }
+  }
+#pragma unroll
+  for (int off = LPR / 2; off >= 1; off >>= 1)
+#pragma unroll
+    for (int t = 0; t < TPL; ++t)
+#pragma unroll
+      for (int h = 0; h < HG; ++h) sc[t][h] += __shfl_xor_sync(0xffffffffu, sc[t][h], off);
+
+  bool valid[TPL];
+#pragma unroll
+  for (int t = 0; t < TPL; ++t) {
+    const int r = rg + t * RPW;
+    valid[t] = r < nvalid && r >= nstart;
+    const float ks = valid[t] ? ksc[r] : 0.f;  // rows outside the range are never read
+#pragma unroll
+    for (int h = 0; h < HG; ++h) sc[t][h] *= ks;
+  }
+  softmax_pv_i8<D, HG, TPL>(st, sc, valid, vp, vsc, rg, sub);
 }
 
 // Merge the row groups of a warp (lanes holding the same D-slice) by

@@ -15,6 +15,7 @@
 
 #include "block_allocator.hpp"
 #include "decode_attn.cuh"
+#include "decode_attn_i8.cuh"
 #include "kv_cache_write.cuh"
 #include "pkv_common.cuh"
 #include "prefill_attn.cuh"
@@ -50,6 +51,40 @@ int device_sm_count(int dev) {
 }
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ------------------------------------------------------------ tensor maps --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// Tiled tensor map; dims/box innermost first, strides in bytes for dims
+// 1..rank-1.  bf16 with a 128-byte swizzle unless told otherwise.
+bool make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+               const cuuint64_t* strides, const cuuint32_t* box,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  return enc(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 
 // ----------------------------------------------------------------- decode --
 constexpr int kDecodeWarps = 4;
@@ -179,6 +214,56 @@ pkv_status launch_decode_any(const pkv::DecodeParams& p, int D, int HG, int B, i
                    : launch_decode_t<64, 1, I8, WIN>(p, B, Hkv, nsub, C, st);
 }
 
+// INT8 cache: Q.K^T on the tensor cores (decode_attn_i8.cuh)
+template <int D, int HG>
+struct DecodeI8Kernel {
+  using S = pkv::DecodeI8Shape<D, HG>;
+  static constexpr auto fn = pkv::decode_attn_i8_kernel<D, HG, false>;
+  static bool prepare(int dev) {
+    static int done[kMaxDevices] = {0};
+    static std::mutex mu;
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> g(mu);
+    if (!done[dev]) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return false;
+      done[dev] = 1;
+    }
+    return true;
+  }
+};
+
+template <int D, int HG>
+pkv_status launch_decode_i8_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C, cudaStream_t st) {
+  using K = DecodeI8Kernel<D, HG>;
+  if (!K::prepare(current_device())) return PKV_ERR_CUDA;
+  // K codes [NB][Hkv][16][D] bytes: one box is one page of one kv head
+  CUtensorMap tm;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)pkv::kPageRows, (cuuint64_t)Hkv, (cuuint64_t)p.NB};
+  const cuuint64_t strides[3] = {(cuuint64_t)D, (cuuint64_t)pkv::kPageRows * D,
+                                 (cuuint64_t)Hkv * pkv::kPageRows * D};
+  const cuuint32_t box[4] = {(cuuint32_t)D, (cuuint32_t)pkv::kPageRows, 1, 1};
+  if (!make_tmap(&tm, p.k_cache, 4, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                 D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+    return PKV_ERR_CUDA;
+  dim3 grid(C, Hkv * nsub, B);
+  K::fn<<<grid, K::S::THREADS, K::S::SMEM_BYTES, st>>>(p, tm);
+  return launch_status();
+}
+
+pkv_status launch_decode_i8(const pkv::DecodeParams& p, int D, int HG, int B, int Hkv, int nsub, int C,
+                            cudaStream_t st) {
+  if (D == 128)
+    return HG == 4 ? launch_decode_i8_t<128, 4>(p, B, Hkv, nsub, C, st)
+           : HG == 2 ? launch_decode_i8_t<128, 2>(p, B, Hkv, nsub, C, st)
+                     : launch_decode_i8_t<128, 1>(p, B, Hkv, nsub, C, st);
+  return HG == 4 ? launch_decode_i8_t<64, 4>(p, B, Hkv, nsub, C, st)
+         : HG == 2 ? launch_decode_i8_t<64, 2>(p, B, Hkv, nsub, C, st)
+                   : launch_decode_i8_t<64, 1>(p, B, Hkv, nsub, C, st);
+}
+
 template <int D>
 pkv_status launch_merge_t(const pkv::MergeParams& mp, int B, int Hq, cudaStream_t st) {
   pkv::lse_merge_kernel<D><<<dim3(Hq, B), D, 0, st>>>(mp);
@@ -197,6 +282,7 @@ pkv_status check_decode_args(void* out, const void* q, const void* k_cache, cons
   if (B == 0) return PKV_OK;
   if (!out || !q || !context_lens || ((MB > 0) && (!block_tables || !k_cache || !v_cache)))
     return PKV_ERR_INVALID_ARG;
+  if (MB > 0 && NB == 0) return PKV_ERR_INVALID_ARG;  // no block a table entry could name
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
   return PKV_OK;
@@ -234,7 +320,7 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
     p.lse_part = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) +
                                           round256(rows * D * sizeof(float)));
   }
-  pkv_status s = k_scale    ? launch_decode_any<true>(p, D, HG, B, Hkv, nsub, C, st)
+  pkv_status s = k_scale    ? launch_decode_i8(p, D, HG, B, Hkv, nsub, C, st)
                  : window > 0 ? launch_decode_any<false, true>(p, D, HG, B, Hkv, nsub, C, st)
                               : launch_decode_any<false>(p, D, HG, B, Hkv, nsub, C, st);
   if (s != PKV_OK) return s;
@@ -259,36 +345,6 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
 }
 
 // ---------------------------------------------------------------- prefill --
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// bf16 tensor map with a 128-byte swizzle; dims/box innermost first, strides
-// in bytes for dims 1..rank-1.
-bool make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-               const cuuint64_t* strides, const cuuint32_t* box) {
-  EncodeTiledFn enc = encode_tiled_fn();
-  if (!enc) return false;
-  const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
-             strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int prefill_prepare(int dev) {
   static int done[kMaxDevices] = {0};
   static std::mutex mu;

@@ -1,5 +1,6 @@
 // tcgen05.cuh -- hand-written PTX wrappers for the sm_100a tensor-core path:
-// tensor-memory (TMEM) allocation, tcgen05.mma (bf16 in, fp32 accumulate),
+// tensor-memory (TMEM) allocation, tcgen05.mma (bf16 in, fp32 accumulate;
+// signed 8-bit in, s32 accumulate),
 // tcgen05.commit onto mbarriers, TMEM loads/stores, and tiled TMA loads.
 //
 // Descriptor bit layouts follow the PTX ISA's tcgen05 "shared memory matrix
@@ -35,13 +36,18 @@ __device__ __forceinline__ void dealloc(uint32_t taddr, uint32_t ncols) {
 }
 
 // ----------------------------------------------------------- descriptors --
-// Shared-memory matrix descriptor, 128-byte swizzle:
+// Shared-memory matrix descriptor of a swizzled K-major (or MN-major) tile:
 //   [0,14) start address >> 4, [16,30) leading byte offset >> 4,
 //   [32,46) stride byte offset >> 4, [46,48) version = 1,
-//   [49,52) base offset = 0, [52] absolute-LBO mode = 0, [61,64) layout = 2.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+//   [49,52) base offset = 0, [52] absolute-LBO mode = 0, [61,64) layout:
+//   2 = 128-byte swizzle, 4 = 64-byte swizzle (the pattern repeats every 8
+//   rows, 1024 or 512 bytes; tiles start on a 1024-byte boundary).
+__device__ __forceinline__ uint64_t smem_desc_sw(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc_sw(saddr, lbo, sbo, 2);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation:
@@ -52,7 +58,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::i8 with signed 8-bit A/B and s32
+// accumulation: [4,6) D format = 2 (s32), [7,10) A format = 1 (s8),
+// [10,13) B format = 1 (s8), both K-major, [17,23) N >> 3, [24,29) M >> 4.
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // -------------------------------------------------------------------- MMA --
+// D[tmem] (+)= A[smem] * B[smem], signed 8-bit operands, s32 accumulator.
+__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]; accumulate = 0 overwrites D.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
@@ -94,6 +118,14 @@ __device__ __forceinline__ void ld_32x32b_x32(uint32_t taddr, uint32_t* r) {
         "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
         "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void ld_32x32b_x8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
 }
 
 __device__ __forceinline__ void st_32x32b_x32(uint32_t taddr, const uint32_t* r) {

@@ -3,7 +3,8 @@
 Cache writes (codes and scales, over the whole pool) must match the oracle
 bit for bit; attention over the int8 pool must satisfy
 |gpu - ref| <= 5e-3 + 1e-2 |ref|, where ref is plain fp64 attention over the
-values code * scale.  Every call goes through the C ABI.
+values code * scale (the kernel holds q as a 15-bit fixed-point pair per head
+for its integer tensor-core scores).  Every call goes through the C ABI.
 """
 import numpy as np
 import pytest
@@ -116,6 +117,24 @@ def test_int8_decode_shapes_and_edges(D, Hq, Hkv):
     out = _decode(case)
     assert_close(out, HostCase(case).decode_ref(), f"int8 D={D} G={Hq // Hkv}")
     assert torch.count_nonzero(out[0]) == 0              # empty context -> zero row
+    assert pkv.get_device_error() == 0
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_int8_decode_query_dynamic_range(D):
+    """Query heads far from unit scale, one dominated by a single element, one
+    all zero: the scores stay within tolerance of plain fp64 attention."""
+    case = _case([5, 77, 300, 1000], 8, 2, D, seed=230 + D)
+    q = case.q.float()
+    q[:, 0] *= 1000.0
+    q[:, 1] *= 1e-3
+    q[:, 2, 0] = 100.0
+    q[:, 3] = 0.0
+    q[:, 4] *= 3e-20
+    q[:, 5] *= 2e15
+    case.q = q.to(torch.bfloat16)
+    out = _decode(case)
+    assert_close(out, HostCase(case).decode_ref(), f"int8 q range D={D}")
     assert pkv.get_device_error() == 0
 
 
