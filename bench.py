@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--profile", default=None,
-                    choices=["decode", "decode_full", "decode_d64", "decode_int8", "split", "prefill", "write"],
+                    choices=["decode", "decode_full", "decode_d64", "decode_int8", "decode_int8_full", "split", "prefill",
+                             "write"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
@@ -403,6 +404,13 @@ def profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
                                 max_context_len=4096)
+    elif kind == "decode_int8_full":
+        # the bench's Llama-3-8B-shaped INT8 decode, full size: 1.1 GB of codes and scales
+        c = wl.workload("llama3_8b_decode_int8", device="cuda")
+        out = torch.empty_like(c.q)
+        for _ in range(launches):
+            pkv.paged_attention_int8(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_tables,
+                                     c.context_lens, c.scale, out=out, max_context_len=4096)
     elif kind == "decode_int8":
         # 32 of the Llama-3-8B-shaped sequences over the INT8 cache: 264 MiB of codes and scales
         c = wl.make_case(B=32, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 32, seed=1006, device="cuda",

@@ -21,11 +21,15 @@
 // One CTA per (split, head group, sequence), 4 consumer warps and one warp
 // that loads and issues the MMAs.  A tile is 8 pages = 128 keys (the MMA's
 // M): their K codes arrive by tiled TMA into 128- (D=128) or 64-byte (D=64)
-// swizzled rows, their V codes and row scales by 1-D bulk copies.  The MMA
+// swizzled rows, their V codes by 1-D bulk copies, their row scales by
+// 16-byte cp.async from the producer warp's lanes.  The MMA
 // writes the tile's scores into one of two TMEM buffers (16 columns each);
 // consumer warp w owns TMEM lanes 32w..32w+31, i.e. the tile's keys
 // 32w..32w+31 (pages 2w, 2w+1), and keeps its own online-softmax state over
-// them, merged across warps at the end as in the CUDA-core kernel.
+// them, merged across warps at the end as in the CUDA-core kernel.  Each
+// lane first takes its own key's weights (one exp per key and head, V scale
+// folded in); then the warp's lanes, 16 elements of D each, accumulate the
+// 32 rows of V codes with those weights.
 #pragma once
 #include <cuda.h>
 
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   if (producer) {
     if (lane == 0) {
       for (int s = 0; s < S::ST; ++s) {
-        mbar_init(full(s), 1);
+        mbar_init(full(s), 1 + 32);  // the bytes of the bulk copies, then one per lane's row scales
         mbar_init(empty(s), S::NW);
       }
       for (int i = 0; i < 2; ++i) {
@@ -224,17 +228,26 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
       const int s = i % S::ST;
       const int np = min(S::TILE_PAGES, n - i * S::TILE_PAGES);
       const int blk = __shfl_sync(0xffffffffu, ent_cur, ((i & 3) << 3) + (lane & 7));
-      if (lane == 0) mbar_arrive_expect_tx(full(s), np * (2 * S::PAGE + 2 * kPageRows * 4));
+      if (lane == 0) mbar_arrive_expect_tx(full(s), np * 2 * S::PAGE);
       __syncwarp();
       if (lane < np) {
         const size_t page = (size_t)blk * p.Hkv + kvh;
         tc::tma_load_4d(base + S::K_OFF + s * S::K_TILE + lane * S::PAGE, &tm_k, 0, 0, kvh, blk, full(s));
         bulk_g2s_hint(base + S::V_OFF + s * S::K_TILE + lane * S::PAGE, p.v_cache + page * S::PAGE, S::PAGE,
                       full(s), pol);
-        const uint32_t sc = base + S::S_OFF + s * S::SC_STAGE + lane * kPageRows * 4;
-        bulk_g2s_hint(sc, p.k_scale + page * kPageRows, kPageRows * 4, full(s), pol);
-        bulk_g2s_hint(sc + S::TILE_ROWS * 4, p.v_scale + page * kPageRows, kPageRows * 4, full(s), pol);
       }
+      // Row scales, 64 bytes per page and pool: as bulk copies they would
+      // double the copies of a tile, and a copy costs about the same whatever
+      // its size, so the 32 lanes gather them 16 bytes each instead.
+      const int pg = lane >> 2;  // page of this lane's two 16-byte pieces
+      const int blk_s = __shfl_sync(0xffffffffu, ent_cur, ((i & 3) << 3) + pg);
+      if (pg < np) {
+        const size_t so = ((size_t)blk_s * p.Hkv + kvh) * kPageRows + (lane & 3) * 4;
+        const uint32_t sc = base + S::S_OFF + s * S::SC_STAGE + lane * 16;
+        cp_async16(sc, p.k_scale + so, pol);
+        cp_async16(sc + S::TILE_ROWS * 4, p.v_scale + so, pol);
+      }
+      cp_async_arrive_noinc(full(s));
     };
     constexpr uint32_t IDESC = tc::idesc_s8_s32(S::TILE_ROWS, S::MMA_N);
     const uint64_t desc_k = tc::smem_desc_sw(base + S::K_OFF, 16, S::SBO, S::SW_LAYOUT);
@@ -313,29 +326,71 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
       const int nvalid = rows_cta - row0, nstart = lo_cta - row0;
       const float* ksc = reinterpret_cast<const float*>(sbase + S::S_OFF + s * S::SC_STAGE) + warp * S::WROWS;
       {
-        // this lane's key: 256 S_hi + S_lo is the exact integer q.k per head
+        // This lane's key.  256 S_hi + S_lo is the exact integer q.k per head.
+        // Its softmax weight is taken here once, not by each lane that
+        // reads the row's V: the running max moves only when a score passes
+        // it by more than 8 (log2), so weights stay below 2^8 and a move,
+        // with its rescale, is rare after the first tile.
         const bool v = lane < nvalid && lane >= nstart;
         const float ks = v ? ksc[lane] : 0.f;  // rows outside the range are never read
+        const float vs = v ? ksc[S::TILE_ROWS + lane] : 0.f;
+        float sc[HG];
+        bool big = false;
+#pragma unroll
+        for (int h = 0; h < HG; ++h) {
+          sc[h] = v ? (float)((int)r[h] * 256 + (int)r[HG + h]) * (ks * cqr[h]) : -INFINITY;
+          big |= sc[h] > st.m[h] + 8.f;
+        }
+        if (__any_sync(0xffffffffu, big)) {
+#pragma unroll
+          for (int h = 0; h < HG; ++h) {
+            float mt = sc[h];
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+            const float mn = fmaxf(st.m[h], mt);
+            const float alpha = (mn == -INFINITY) ? 1.f : ex2(st.m[h] - mn);
+            st.m[h] = mn;
+            st.l[h] *= alpha;
+            const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) st.acc[h][e] = __fmul2_rn(st.acc[h][e], a2);
+          }
+        }
         float o[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h)
-          o[h] = h < HG ? (float)((int)r[h] * 256 + (int)r[HG + h]) * (ks * cqr[h]) : 0.f;
+        for (int h = 0; h < 4; ++h) {
+          if (h < HG) {
+            const float pr = v ? ex2(sc[h] - st.m[h]) : 0.f;
+            st.l[h] += pr;      // this lane's keys only; summed over the warp at the end
+            o[h] = pr * vs;     // the V scale rides on the weight
+          } else {
+            o[h] = 0.f;
+          }
+        }
         *reinterpret_cast<float4*>(scw + lane * 4) = make_float4(o[0], o[1], o[2], o[3]);
       }
       __syncwarp();
-      float sc[TPL][HG];
-      bool valid[TPL];
+      // every row of the warp's slice: invalid rows carry weight 0 and their
+      // codes are finite bytes, so no row needs a test
+      const unsigned char* vp = sbase + S::V_OFF + s * S::K_TILE + warp * S::WROWS * D;
 #pragma unroll
       for (int t = 0; t < TPL; ++t) {
         const int rr = rg + t * RPW;
-        valid[t] = rr < nvalid && rr >= nstart;
-        const float4 v4 = *reinterpret_cast<const float4*>(scw + rr * 4);
-        const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+        const float4 w4 = *reinterpret_cast<const float4*>(scw + rr * 4);
+        const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+        const uint4 va = reinterpret_cast<const uint4*>(vp + rr * D)[sub];
+        float2 v2[8];
+        widen_i8x4(va.x, v2[0], v2[1]);
+        widen_i8x4(va.y, v2[2], v2[3]);
+        widen_i8x4(va.z, v2[4], v2[5]);
+        widen_i8x4(va.w, v2[6], v2[7]);
 #pragma unroll
-        for (int h = 0; h < HG; ++h) sc[t][h] = vv[h];
+        for (int h = 0; h < HG; ++h) {
+          const float2 pp = make_float2(wv[h], wv[h]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) st.acc[h][e] = __ffma2_rn(pp, v2[e], st.acc[h][e]);
+        }
       }
-      softmax_pv_i8<D, HG, TPL>(st, sc, valid, sbase + S::V_OFF + s * S::K_TILE + warp * S::WROWS * D,
-                                ksc + S::TILE_ROWS, rg, sub);
       // the stage is refilled by the copy engine after this: order the reads first
       fence_proxy_async_smem();
       __syncwarp();
@@ -350,6 +405,15 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
     tc::fence_after_sync();
     tc::dealloc(tmem, S::TMEM_COLS);
   } else {
+    // the running max is the warp's; the sums are per key lane: total them,
+    // held once per column of lanes so the row-group merge adds them once
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      float l = st.l[h];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+      st.l[h] = rg == 0 ? l : 0.f;
+    }
     warp_merge<D, HG, false>(st);
     warp_store<D, HG>(reinterpret_cast<float*>(sbase + S::K_OFF) + warp * S::MERGE_STRIDE, st, rg, sub,
                       2 * sub, 2 * sub + 1);

@@ -107,6 +107,19 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return pol;
 }
 
+// 16-byte asynchronous copy global -> shared through L2 only (dst and src
+// 16-byte aligned); completion is reported by cp_async_arrive_noinc.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(policy)
+               : "memory");
+}
+
+// One arrival on `bar` once every cp.async this thread issued before has
+// landed; the arrival is part of the barrier's initial count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes,
                                               uint32_t bar, uint64_t policy) {
   asm volatile(
