@@ -234,7 +234,8 @@ class OracleSample:
     def describe(self, reps: int, secs: float) -> str:
         sp = self.spec
         return (f"fp64 C oracle decode of {self.n} of the {sp['B']} sequences (ctx {sp['lens'][0]}, "
-                f"{sp['Hq']} q / {sp['Hkv']} kv heads, D={sp['D']}) x {reps}, OpenMP, {secs:.1f} s")
+                f"{sp['Hq']} q / {sp['Hkv']} kv heads, D={sp['D']}) x {reps}, OpenMP on "
+                f"{self.orc.num_threads()} threads, {secs:.1f} s")
 
 
 def oracle_decode_rate(seconds: float):
@@ -304,10 +305,51 @@ def time_calls(fn, iters, flush=None):
     return [e0.elapsed_time(e1) for e0, e1 in ev]
 
 
-def extras(peaks):
+def timed_us(fn, iters=50, flush=None):
+    time_calls(fn, 3, flush)
+    return statistics.median(time_calls(fn, iters, flush)) * 1e3
+
+
+def extras(peaks, decode_gbs):
     import paged_kv_cache_477_b200 as pkv
     from paged_kv_cache_477_b200 import workloads as wl
     res = {}
+    # read-only HBM stream (what decode does: reads K/V, writes ~nothing), 4 GiB
+    buf = torch.empty(4 << 30, dtype=torch.uint8, device="cuda")
+    sink = torch.empty(torch.cuda.get_device_properties(0).multi_processor_count * 2, dtype=torch.int32,
+                       device="cuda")  # two CTAs per SM, 96 KB of chunks in flight each
+    by_chunk = {}
+    for chunk in (32768, 16384, 8192, 4096):
+        us = timed_us(lambda: pkv.hbm_read_probe(buf, sink, chunk), 10)
+        by_chunk[chunk] = buf.numel() / (us * 1e-6) / 1e9
+    probe = max(by_chunk.values())
+    res["hbm_read_probe"] = {"GB/s": round(probe, 1), "bytes": buf.numel(),
+                             "GB/s_by_copy_bytes": {str(k): round(v, 1) for k, v in by_chunk.items()},
+                             "in_flight": "96 KB per CTA, 2 CTAs per SM",
+                             "headline_decode_frac_of_probe": round(decode_gbs / probe, 4),
+                             "headline_decode_frac_of_8tbs_nominal": round(decode_gbs / 8000.0, 4)}
+    del buf, sink
+    torch.cuda.empty_cache()
+    # the tiny parity case, warm (latency only)
+    c = wl.workload("tiny_decode", device="cuda")
+    us = timed_us(lambda: pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens,
+                                              c.scale))
+    res["tiny_decode"] = {"us": round(us, 2), "l2": "warm (70 KB of K/V)"}
+    # cache writes of the headline step (128 new rows), plain and with RoPE on K
+    c = wl.workload(WORKLOAD, device="cuda")
+    T = c.new_key.shape[0]
+    pos = c.context_lens.to(torch.int64) - 1
+    for name, fn, nb in (
+            ("kv_cache_write_128", lambda: pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache,
+                                                              c.slot_mapping), write_bytes(c)),
+            ("kv_cache_write_rope_128", lambda: pkv.kv_cache_write_rope(c.new_key, c.new_value, c.k_cache,
+                                                                        c.v_cache, c.slot_mapping, pos, 500000.0),
+             write_bytes(c) + 8 * T)):
+        us = timed_us(fn)
+        res[name] = {"us": round(us, 2), "GB/s": round(nb / (us * 1e-6) / 1e9, 1), "tokens": T, "bytes": nb,
+                     "l2": "new rows warm in L2; rows scattered into a 2 GiB pool"}
+    del c
+    torch.cuda.empty_cache()
     for name, hint in (("llama32_1b_decode", 4096), ("ragged_long_decode", 32768)):
         c = wl.workload(name, device="cuda")
         out = torch.empty_like(c.q)
@@ -358,10 +400,21 @@ def extras(peaks):
                                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "launches": pkv.last_launch_count(),
                                     "bytes": decode_bytes(c), "kv_bytes_vs_bf16": 0.5 + 2.0 / c.D,
                                     "l2": "inputs larger than L2"}
+    T = c.new_key.shape[0]
+    nb = 2 * T * c.Hkv * c.D * 2 + 2 * T * c.Hkv * (c.D + 4) + 8 * T
+    us = timed_us(lambda: pkv.kv_cache_write_int8(c.new_key, c.new_value, c.k_cache, c.v_cache, c.k_scale,
+                                                  c.v_scale, c.slot_mapping))
+    res["kv_cache_write_int8_128"] = {"us": round(us, 2), "GB/s": round(nb / (us * 1e-6) / 1e9, 1), "tokens": T,
+                                      "bytes": nb, "l2": "new rows warm in L2; rows scattered into the int8 pool"}
     del c, out, ws
     torch.cuda.empty_cache()
     c = wl.workload("chunked_prefill", device="cuda")
-    pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)
+    # the prefill's pre-step: the chunk's 2048 rows into the cache
+    wfn = lambda: pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)
+    us = timed_us(wfn)
+    res["kv_cache_write_2048"] = {"us": round(us, 2), "GB/s": round(write_bytes(c) / (us * 1e-6) / 1e9, 1),
+                                  "tokens": c.new_key.shape[0], "bytes": write_bytes(c),
+                                  "l2": "new rows warm in L2"}
     out = torch.empty_like(c.q)
     fn = lambda: pkv.paged_attention_prefill(c.q, c.query_start_loc, c.k_cache, c.v_cache, c.block_tables,
                                              c.context_lens, c.scale, c.max_q_len, out=out)
@@ -373,7 +426,11 @@ def extras(peaks):
         tf = prefill_flops(c) / (ms * 1e-3) / 1e12
         res["chunked_prefill"] = {"TFLOP/s": round(tf, 1), "us": round(ms * 1e3, 2),
                                   "frac_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+                                  "frac_bf16_nominal_2250": round(tf / 2250.0, 4),
                                   "flops": prefill_flops(c), "l2": "flushed (256 MiB write) before each call"}
+        us = timed_us(fn, 20)
+        res["chunked_prefill_warm"] = {"TFLOP/s": round(prefill_flops(c) / (us * 1e-6) / 1e12, 1),
+                                       "us": round(us, 2), "l2": "warm (no flush between calls)"}
     except pkv.PagedKVError as e:
         res["chunked_prefill"] = {"unavailable": str(e)}
     return res
@@ -577,11 +634,17 @@ def main():
             "clocks": clocks,
         }
         if not args.no_extras and world == 1:
-            line["extras"] = extras(peaks)
+            line["extras"] = extras(peaks, achieved)
         if world == 1:
             v, cores, desc = oracle_decode_rate(args.cpu_seconds)
             line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                                     "sample": desc}
+            if "extras" in line:
+                import oracle
+                oracle.get().set_num_threads(1)
+                v1, _, desc1 = oracle_decode_rate(min(4.0, args.cpu_seconds))
+                oracle.get().set_num_threads(cores)
+                line["extras"]["oracle_one_core"] = {"value": round(v1, 4), "unit": "GB/s", "sample": desc1}
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

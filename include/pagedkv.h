@@ -345,6 +345,20 @@ int32_t pkv_block_allocator_num_free(pkv_block_allocator* a);
 int32_t pkv_block_allocator_refcount(pkv_block_allocator* a, int32_t id);
 
 /*
+ * hbm_read_probe -- measurement utility, not part of the attention path:
+ * reads `bytes` (a multiple of 16) of device memory at `buf` (16-byte
+ * aligned) once, in chunks of chunk_bytes moved by bulk copies into shared
+ * memory (as decode moves pages), 96 KB in flight per CTA, chunk c by CTA
+ * c % nsink.  chunk_bytes divides 98304 and lies in [4096, 32768].  CTA i
+ * writes to sink[i] (device, nsink words) the XOR of the first four 32-bit
+ * words of each of its chunks.  Timed by the caller, it gives the read-only
+ * bandwidth that HBM-bound decode is compared with, and how it depends on
+ * the size of each copy.  One launch.
+ */
+pkv_status pkv_hbm_read_probe(const void* buf, size_t bytes, int32_t chunk_bytes, uint32_t* sink,
+                              int32_t nsink, pkv_stream_t stream);
+
+/*
  * copy_blocks -- for each (src, dst) pair in `pairs` (device, [n][2] int32)
  * copy block src to block dst, bit for bit, in both pools (k_cache and
  * v_cache; for the INT8 cache call once for the codes and once for the

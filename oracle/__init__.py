@@ -73,6 +73,8 @@ class Oracle:
         self.path = path
         lib = ctypes.CDLL(path)
         lib.ref_num_threads.restype = ctypes.c_int
+        lib.ref_set_num_threads.argtypes = [ctypes.c_int]
+        lib.ref_set_num_threads.restype = None
         lib.ref_mutant_id.restype = ctypes.c_int
         lib.ref_kv_cache_write.argtypes = [_P, _P, _I64, _I64, _P, _P, _P, _I32, _I32, _I32, _I32, _I32]
         lib.ref_paged_attention.argtypes = [_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32]
@@ -103,6 +105,9 @@ class Oracle:
 
     def num_threads(self) -> int:
         return int(self.lib.ref_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.ref_set_num_threads(int(n))
 
     @staticmethod
     def _check(rc: int, what: str, allow_bounds: bool = False) -> int:

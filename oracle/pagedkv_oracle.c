@@ -74,6 +74,15 @@ int ref_num_threads(void) {
 #endif
 }
 
+/* Threads the next parallel loops use (timing on one core or all). */
+void ref_set_num_threads(int n) {
+#ifdef _OPENMP
+  omp_set_num_threads(n > 0 ? n : 1);
+#else
+  (void)n;
+#endif
+}
+
 int ref_mutant_id(void) { return PKV_ORACLE_MUTANT; }
 
 /* ------------------------------------------------------------------------- */

@@ -77,6 +77,7 @@ EXPORTS = {
     "pkv_block_allocator_num_free": ([_P], _I32),
     "pkv_block_allocator_refcount": ([_P, _I32], _I32),
     "pkv_copy_blocks": ([_P, _P, _SZ, _P, _I32, _I32, _P], _I32),
+    "pkv_hbm_read_probe": ([_P, _SZ, _I32, _P, _I32, _P], _I32),
     "pkv_get_device_error": ([_P, ctypes.POINTER(_I32)], _I32),
     "pkv_last_launch_count": ([], _I32),
     "pkv_status_string": ([_I32], ctypes.c_char_p),
@@ -476,6 +477,16 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, pairs: torch.Tenso
     rc = load_library().pkv_copy_blocks(k_cache.data_ptr(), v_cache.data_ptr(), k_cache[0].nbytes,
                                         pairs.data_ptr(), pairs.shape[0], k_cache.shape[0], _stream(stream))
     _check(rc, "copy_blocks")
+
+
+def hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, chunk_bytes: int = 32768, stream=None) -> None:
+    """Read all of `buf` once in bulk copies of `chunk_bytes` (measurement
+    utility); one uint32 per CTA into `sink`."""
+    _contig(_dev(buf, "buf"), "buf")
+    _contig(_dev(sink, "sink", torch.int32), "sink")
+    rc = load_library().pkv_hbm_read_probe(buf.data_ptr(), buf.numel() * buf.element_size(), int(chunk_bytes),
+                                           sink.data_ptr(), sink.numel(), _stream(stream))
+    _check(rc, "hbm_read_probe")
 
 
 def get_device_error(stream=None) -> int:

@@ -31,7 +31,8 @@ def nvcc_path() -> str:
 
 
 def _deps():
-    return [SRC] + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "pagedkv.h")]
+    return ([SRC] + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.hpp")) +
+            [os.path.join(ROOT, "include", "pagedkv.h")])
 
 
 def up_to_date() -> bool:

@@ -72,21 +72,16 @@ __device__ __forceinline__ int window_first_key(int L, int window) {
 }
 
 // A ring stage holds PPS consecutive pages of one sequence: their K pages
-// side by side (ROWS = 16 * PPS contiguous key rows), then their V pages;
-// for the int8 cache (I8) then the pages' K scales and V scales (16 fp32 per
-// page each).
-template <int D, int HG, int NW, int SW, int PPS, bool I8 = false>
+// side by side (ROWS = 16 * PPS contiguous key rows), then their V pages.
+template <int D, int HG, int NW, int SW, int PPS>
 struct DecodeShape {
   static_assert(D == 64 || D == 128, "head_dim");
   static constexpr int LPR = D / 16;              // lanes sharing one key row
   static constexpr int RPW = 32 / LPR;            // rows per warp step
   static constexpr int ROWS = kPageRows * PPS;    // key rows per stage
   static constexpr int TPL = ROWS / RPW;          // rows per lane per stage
-  static constexpr int PAGE_BYTES = kPageRows * D * (I8 ? 1 : 2);
-  static constexpr int SCALE_BYTES = I8 ? kPageRows * 4 : 0;  // per page, K or V
-  static constexpr int KS_OFF = 2 * PPS * PAGE_BYTES;         // K scales within a stage
-  static constexpr int VS_OFF = KS_OFF + PPS * SCALE_BYTES;   // V scales
-  static constexpr int STAGE_BYTES = 2 * PPS * (PAGE_BYTES + SCALE_BYTES);
+  static constexpr int PAGE_BYTES = kPageRows * D * 2;
+  static constexpr int STAGE_BYTES = 2 * PPS * PAGE_BYTES;
   static constexpr int THREADS = NW * 32;
   static constexpr int WARP_RING = SW * STAGE_BYTES;
   static constexpr int RING_BYTES = NW * WARP_RING;
@@ -211,13 +206,9 @@ __device__ __forceinline__ void attend_rows(LaneState<HG>& st, const float2 (&q2
   }
 }
 
-// INT8 cache: ROWS key rows of int8 codes (K at kp, V at vp, row stride D
-// bytes) with one fp32 scale per row (ksc, vsc).  The lane holds the 16
-// consecutive elements [16 * sub, 16 * sub + 16) of its rows (q2 in that
-// order).  A code c becomes a float exactly as (2^23 + (c + 128)) - (2^23 +
-// 128): a byte permute builds the first term's bit pattern, one packed
-// subtract finishes.  The K scale multiplies the reduced dot product; the V
-// scale multiplies the probability, so neither touches the 16-wide inner loops.
+// Four int8 codes (one 32-bit word) to four exact floats: a code c becomes
+// (2^23 + (c + 128)) - (2^23 + 128); a byte permute builds the first term's
+// bit pattern, one packed subtract finishes.
 __device__ __forceinline__ void widen_i8x4(uint32_t w, float2& lo, float2& hi) {
   const uint32_t x = w ^ 0x80808080u;  // biased codes c + 128
   const float2 bias = make_float2(-8388736.f, -8388736.f);
@@ -225,103 +216,6 @@ __device__ __forceinline__ void widen_i8x4(uint32_t w, float2& lo, float2& hi) {
                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7541))), bias);
   hi = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7542)),
                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7543))), bias);
-}
-
-// Online softmax and P.V over TPL rows of int8 V codes (row stride D bytes,
-// one fp32 scale per row in vsc): sc[t][h] are the rows' scores (log2
-// domain), valid[t] whether row rg + t * RPW takes part.  Invalid rows take no
-// part in the max and are never read from V.
-template <int D, int HG, int TPL>
-__device__ __forceinline__ void softmax_pv_i8(LaneState<HG>& st, const float (&sc)[TPL][HG],
-                                              const bool (&valid)[TPL], const unsigned char* vp,
-                                              const float* vsc, int rg, int sub) {
-  constexpr int RPW = 32 / (D / 16);
-  float mp[HG];
-  bool grow = false;
-#pragma unroll
-  for (int h = 0; h < HG; ++h) {
-    mp[h] = -INFINITY;
-#pragma unroll
-    for (int t = 0; t < TPL; ++t)
-      if (valid[t]) mp[h] = fmaxf(mp[h], sc[t][h]);
-    grow |= mp[h] > st.m[h];
-  }
-  if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      const float mn = fmaxf(st.m[h], mp[h]);
-      const float alpha = (mn == -INFINITY) ? 1.f : ex2(st.m[h] - mn);
-      st.m[h] = mn;
-      st.l[h] *= alpha;
-      const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) st.acc[h][e] = __fmul2_rn(st.acc[h][e], a2);
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    if (!valid[t]) continue;
-    const int r = rg + t * RPW;
-    const uint4 va = reinterpret_cast<const uint4*>(vp + r * D)[sub];
-    float2 v2[8];
-    widen_i8x4(va.x, v2[0], v2[1]);
-    widen_i8x4(va.y, v2[2], v2[3]);
-    widen_i8x4(va.z, v2[4], v2[5]);
-    widen_i8x4(va.w, v2[6], v2[7]);
-    const float vs = vsc[r];
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      const float pr = ex2(sc[t][h] - st.m[h]);
-      st.l[h] += pr;
-      const float pv = pr * vs;
-      const float2 pp = make_float2(pv, pv);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) st.acc[h][e] = __ffma2_rn(pp, v2[e], st.acc[h][e]);
-    }
-  }
-}
-
-template <int D, int HG, int ROWS>
-__device__ __forceinline__ void attend_rows_i8(LaneState<HG>& st, const float2 (&q2)[HG][8],
-                                               const unsigned char* kp, const unsigned char* vp,
-                                               const float* ksc, const float* vsc, int nstart, int nvalid,
-                                               int rg, int sub) {
-  constexpr int LPR = D / 16, RPW = 32 / LPR, TPL = ROWS / RPW;
-  float sc[TPL][HG];
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    const int r = rg + t * RPW;
-    const uint4 ka = reinterpret_cast<const uint4*>(kp + r * D)[sub];
-    float2 k2[8];
-    widen_i8x4(ka.x, k2[0], k2[1]);
-    widen_i8x4(ka.y, k2[2], k2[3]);
-    widen_i8x4(ka.z, k2[4], k2[5]);
-    widen_i8x4(ka.w, k2[6], k2[7]);
-#pragma unroll
-    for (int h = 0; h < HG; ++h) {
-      float2 d = __fmul2_rn(q2[h][0], k2[0]);
-#pragma unroll
-      for (int e = 1; e < 8; ++e) d = __ffma2_rn(q2[h][e], k2[e], d);
-      sc[t][h] = d.x + d.y;
-    }
-  }
-#pragma unroll
-  for (int off = LPR / 2; off >= 1; off >>= 1)
-#pragma unroll
-    for (int t = 0; t < TPL; ++t)
-#pragma unroll
-      for (int h = 0; h < HG; ++h) sc[t][h] += __shfl_xor_sync(0xffffffffu, sc[t][h], off);
-
-  bool valid[TPL];
-#pragma unroll
-  for (int t = 0; t < TPL; ++t) {
-    const int r = rg + t * RPW;
-    valid[t] = r < nvalid && r >= nstart;
-    const float ks = valid[t] ? ksc[r] : 0.f;  // rows outside the range are never read
-#pragma unroll
-    for (int h = 0; h < HG; ++h) sc[t][h] *= ks;
-  }
-  softmax_pv_i8<D, HG, TPL>(st, sc, valid, vp, vsc, rg, sub);
 }
 
 // Merge the row groups of a warp (lanes holding the same D-slice) by
@@ -420,10 +314,10 @@ __device__ __forceinline__ void drain_ring(uint32_t wbar, int issued) {
 // ============================================================================
 // One CTA per (split, head group, sequence).
 // ============================================================================
-template <int D, int HG, int NW, int SW, int PPS, bool I8 = false, bool WIN = false>
+template <int D, int HG, int NW, int SW, int PPS, bool WIN = false>
 __global__ void __launch_bounds__(NW * 32)
     decode_attn_kernel(const __grid_constant__ DecodeParams p) {
-  using S = DecodeShape<D, HG, NW, SW, PPS, I8>;
+  using S = DecodeShape<D, HG, NW, SW, PPS>;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int split = blockIdx.x, hsub = blockIdx.y, b = blockIdx.z;
@@ -520,18 +414,13 @@ __global__ void __launch_bounds__(NW * 32)
     if (lane == 0) {
       const int s = k % SW;
       const uint32_t stage = wring + s * S::STAGE_BYTES;
-      mbar_arrive_expect_tx(wbar + 8 * s, np * 2 * (S::PAGE_BYTES + S::SCALE_BYTES));
+      mbar_arrive_expect_tx(wbar + 8 * s, np * 2 * S::PAGE_BYTES);
 #pragma unroll
       for (int i = 0; i < PPS; ++i) {
         if (i >= np) break;
         const size_t off = ((size_t)blk[i] * p.Hkv + kvh) * S::PAGE_BYTES;
         bulk_g2s_hint(stage + i * S::PAGE_BYTES, p.k_cache + off, S::PAGE_BYTES, wbar + 8 * s, pol);
         bulk_g2s_hint(stage + (PPS + i) * S::PAGE_BYTES, p.v_cache + off, S::PAGE_BYTES, wbar + 8 * s, pol);
-        if constexpr (I8) {  // the page's 16 row scales, 64 bytes each for K and V
-          const size_t so = ((size_t)blk[i] * p.Hkv + kvh) * kPageRows;
-          bulk_g2s_hint(stage + S::KS_OFF + i * S::SCALE_BYTES, p.k_scale + so, S::SCALE_BYTES, wbar + 8 * s, pol);
-          bulk_g2s_hint(stage + S::VS_OFF + i * S::SCALE_BYTES, p.v_scale + so, S::SCALE_BYTES, wbar + 8 * s, pol);
-        }
       }
     }
     ++issued;
@@ -543,9 +432,9 @@ __global__ void __launch_bounds__(NW * 32)
   // bf16: the lane's two 16-byte vectors of a row (D=64 odd row groups in
   // swapped order); int8: its 16 consecutive elements, i.e. bf16 vectors
   // 2 * sub and 2 * sub + 1 of q and of the output
-  const int swap = (D == 64 && !I8) ? (rg & 1) : 0;
-  const int ch0 = I8 ? 2 * sub : sub + S::LPR * swap;           // 16-byte bf16 vector held in slot 0
-  const int ch1 = I8 ? 2 * sub + 1 : sub + S::LPR * (swap ^ 1);  // and in slot 1
+  const int swap = D == 64 ? (rg & 1) : 0;
+  const int ch0 = sub + S::LPR * swap;        // 16-byte vector held in slot 0
+  const int ch1 = sub + S::LPR * (swap ^ 1);  // and in slot 1
   float2 q2[HG][8];
   load_q<D, HG>(q2, p.q + ((size_t)b * p.Hq + head0) * D, ch0, ch1, p.scale_log2);
   LaneState<HG> st;
@@ -564,15 +453,8 @@ __global__ void __launch_bounds__(NW * 32)
     const bool ok = mbar_wait(wbar + 8 * s, (j / SW) & 1);
     if (!__all_sync(0xffffffffu, ok)) break;
     const unsigned char* kp = wring_ptr + s * S::STAGE_BYTES;
-    if constexpr (I8)
-      attend_rows_i8<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES,
-                                     reinterpret_cast<const float*>(kp + S::KS_OFF),
-                                     reinterpret_cast<const float*>(kp + S::VS_OFF),
-                                     lo_cta - (warp + j * NW) * S::ROWS, rows_cta - (warp + j * NW) * S::ROWS, rg,
-                                     sub);
-    else
-      attend_rows<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES, lo_cta - (warp + j * NW) * S::ROWS,
-                                  rows_cta - (warp + j * NW) * S::ROWS, rg, ch0, ch1);
+    attend_rows<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES, lo_cta - (warp + j * NW) * S::ROWS,
+                                rows_cta - (warp + j * NW) * S::ROWS, rg, ch0, ch1);
     if (issued < my_n) {
       // the stage just read is refilled: order the generic-proxy reads of all
       // lanes before the copy engine's writes
@@ -586,7 +468,7 @@ __global__ void __launch_bounds__(NW * 32)
   if (done < issued && lane == 0) drain_ring<SW>(wbar, issued);
   __syncwarp();
 
-  warp_merge<D, HG, (D == 64 && !I8)>(st);
+  warp_merge<D, HG>(st);
   // after its last page a warp reuses its own ring for its merge data
   warp_store<D, HG>(reinterpret_cast<float*>(wring_ptr), st, rg, sub, ch0, ch1);
   __syncthreads();

@@ -85,7 +85,8 @@ template <int D, int HG, bool WIN = false>
 __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
     decode_attn_i8_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tm_k) {
   using S = DecodeI8Shape<D, HG>;
-  extern __shared__ __align__(128) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_i8[];
+  unsigned char* smem_raw = smem_i8;
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   unsigned char* sbase = smem_raw + (base - raw_addr);

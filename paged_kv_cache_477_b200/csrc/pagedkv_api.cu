@@ -16,6 +16,7 @@
 #include "block_allocator.hpp"
 #include "decode_attn.cuh"
 #include "decode_attn_i8.cuh"
+#include "hbm_probe.cuh"
 #include "kv_cache_write.cuh"
 #include "pkv_common.cuh"
 #include "prefill_attn.cuh"
@@ -88,21 +89,19 @@ bool make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* d
 
 // ----------------------------------------------------------------- decode --
 constexpr int kDecodeWarps = 4;
-// pages per ring stage: one 8 KB bf16 page pair at D=128, otherwise two, so a
-// stage is 32 key rows whenever a page is smaller and a lane always works on
-// four rows per step
-constexpr int pages_per_stage(int D, bool I8) { return (D == 128 && !I8) ? 1 : 2; }
-// stages per warp: ~96-104 KB of pages in flight per CTA, two CTAs per SM
-// (3 x 8 KB bf16, 3 x 8.25 KB int8 at D=128, 6 x 4.25 KB int8 at D=64)
-constexpr int stages_for(int D, bool I8) { return (I8 && D == 64) ? 6 : 3; }
+// pages per ring stage: one 8 KB page pair at D=128, two at D=64, so a stage
+// is 32 key rows whenever a page is smaller and a lane always works on four
+// rows per step
+constexpr int pages_per_stage(int D) { return D == 128 ? 1 : 2; }
+// stages per warp: 96 KB of pages in flight per CTA, two CTAs per SM
+constexpr int kDecodeStages = 3;
 
-template <int D, int HG, bool I8 = false>
-using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, stages_for(D, I8), pages_per_stage(D, I8), I8>;
+template <int D, int HG>
+using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D)>;
 
-template <int D, int HG, bool I8 = false, bool WIN = false>
+template <int D, int HG, bool WIN = false>
 struct DecodeKernel {
-  static constexpr auto fn =
-      pkv::decode_attn_kernel<D, HG, kDecodeWarps, stages_for(D, I8), pages_per_stage(D, I8), I8, WIN>;
+  static constexpr auto fn = pkv::decode_attn_kernel<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D), WIN>;
   // set the dynamic shared-memory limit once per device; return CTAs per SM
   static int prepare(int dev) {
     static int occ[kMaxDevices] = {0};
@@ -110,14 +109,14 @@ struct DecodeKernel {
     if (dev < 0 || dev >= kMaxDevices) return 1;
     std::lock_guard<std::mutex> g(mu);
     if (occ[dev] == 0) {
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               DecodeS<D, HG, I8>::SMEM_BYTES) != cudaSuccess ||
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeS<D, HG>::SMEM_BYTES) !=
+              cudaSuccess ||
           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return -1;
       int n = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DecodeS<D, HG, I8>::THREADS,
-                                                        DecodeS<D, HG, I8>::SMEM_BYTES) != cudaSuccess ||
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DecodeS<D, HG>::THREADS,
+                                                        DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess ||
           n <= 0)
         return -1;
       occ[dev] = n;
@@ -192,26 +191,25 @@ DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, 
   return pl;
 }
 
-template <int D, int HG, bool I8 = false, bool WIN = false>
-pkv_status launch_decode_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C,
-                           cudaStream_t st) {
-  using K = DecodeKernel<D, HG, I8, WIN>;
+template <int D, int HG, bool WIN = false>
+pkv_status launch_decode_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C, cudaStream_t st) {
+  using K = DecodeKernel<D, HG, WIN>;
   if (K::prepare(current_device()) < 0) return PKV_ERR_CUDA;
   dim3 grid(C, Hkv * nsub, B);
-  K::fn<<<grid, DecodeS<D, HG, I8>::THREADS, DecodeS<D, HG, I8>::SMEM_BYTES, st>>>(p);
+  K::fn<<<grid, DecodeS<D, HG>::THREADS, DecodeS<D, HG>::SMEM_BYTES, st>>>(p);
   return launch_status();
 }
 
-template <bool I8, bool WIN = false>
+template <bool WIN>
 pkv_status launch_decode_any(const pkv::DecodeParams& p, int D, int HG, int B, int Hkv, int nsub, int C,
                              cudaStream_t st) {
   if (D == 128)
-    return HG == 4 ? launch_decode_t<128, 4, I8, WIN>(p, B, Hkv, nsub, C, st)
-           : HG == 2 ? launch_decode_t<128, 2, I8, WIN>(p, B, Hkv, nsub, C, st)
-                     : launch_decode_t<128, 1, I8, WIN>(p, B, Hkv, nsub, C, st);
-  return HG == 4 ? launch_decode_t<64, 4, I8, WIN>(p, B, Hkv, nsub, C, st)
-         : HG == 2 ? launch_decode_t<64, 2, I8, WIN>(p, B, Hkv, nsub, C, st)
-                   : launch_decode_t<64, 1, I8, WIN>(p, B, Hkv, nsub, C, st);
+    return HG == 4 ? launch_decode_t<128, 4, WIN>(p, B, Hkv, nsub, C, st)
+           : HG == 2 ? launch_decode_t<128, 2, WIN>(p, B, Hkv, nsub, C, st)
+                     : launch_decode_t<128, 1, WIN>(p, B, Hkv, nsub, C, st);
+  return HG == 4 ? launch_decode_t<64, 4, WIN>(p, B, Hkv, nsub, C, st)
+         : HG == 2 ? launch_decode_t<64, 2, WIN>(p, B, Hkv, nsub, C, st)
+                   : launch_decode_t<64, 1, WIN>(p, B, Hkv, nsub, C, st);
 }
 
 // INT8 cache: Q.K^T on the tensor cores (decode_attn_i8.cuh)
@@ -321,7 +319,7 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
                                           round256(rows * D * sizeof(float)));
   }
   pkv_status s = k_scale    ? launch_decode_i8(p, D, HG, B, Hkv, nsub, C, st)
-                 : window > 0 ? launch_decode_any<false, true>(p, D, HG, B, Hkv, nsub, C, st)
+                 : window > 0 ? launch_decode_any<true>(p, D, HG, B, Hkv, nsub, C, st)
                               : launch_decode_any<false>(p, D, HG, B, Hkv, nsub, C, st);
   if (s != PKV_OK) return s;
   int launches = 1;
@@ -610,6 +608,33 @@ pkv_status pkv_block_allocator_cow(pkv_block_allocator* a, int32_t id, int32_t* 
 int32_t pkv_block_allocator_num_free(pkv_block_allocator* a) { return a ? a->impl.num_free() : -1; }
 
 int32_t pkv_block_allocator_refcount(pkv_block_allocator* a, int32_t id) { return a ? a->impl.refcount(id) : -1; }
+
+pkv_status pkv_hbm_read_probe(const void* buf, size_t bytes, int32_t chunk_bytes, uint32_t* sink, int32_t nsink,
+                              pkv_stream_t stream) {
+  t_launches = 0;
+  if (!buf || !sink || nsink <= 0 || bytes == 0 || bytes % 16 != 0 || !aligned16(buf))
+    return PKV_ERR_INVALID_ARG;
+  if (chunk_bytes < 4096 || chunk_bytes > pkv::kProbeRing / 3 || pkv::kProbeRing % chunk_bytes != 0)
+    return PKV_ERR_INVALID_ARG;
+  {
+    static int ready[kMaxDevices] = {0};
+    static std::mutex mu;
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return PKV_ERR_CUDA;
+    std::lock_guard<std::mutex> g(mu);
+    if (!ready[dev]) {
+      if (cudaFuncSetAttribute(pkv::hbm_read_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               pkv::kProbeSmem) != cudaSuccess)
+        return PKV_ERR_CUDA;
+      ready[dev] = 1;
+    }
+  }
+  pkv::hbm_read_probe_kernel<<<nsink, 32, pkv::kProbeSmem, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const unsigned char*>(buf), (int64_t)bytes, chunk_bytes, sink);
+  pkv_status s = launch_status();
+  if (s == PKV_OK) t_launches = 1;
+  return s;
+}
 
 pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, size_t block_bytes, const int32_t* pairs, int32_t n,
                            int32_t NB, pkv_stream_t stream) {
