@@ -116,7 +116,7 @@ EDGE_LENS = [0, 1, 15, 16, 17, 31, 32, 33, 100, 257, 600]
 
 
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2), (8, 2), (16, 2), (6, 2), (32, 8)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2), (8, 2), (16, 2), (6, 2), (32, 8), (16, 8), (24, 12), (8, 8)])
 def test_decode_shapes_and_edges(D, Hq, Hkv):
     case = _decode_case(EDGE_LENS, Hq, Hkv, D, seed=100 + D + Hq)
     host = HostCase(case)
@@ -184,8 +184,9 @@ def test_split_count_invariance():
         assert d <= 2 * (5e-3 + 1e-2 * outs[0].float().abs().max().item())
 
 
-def test_decode_bad_block_id_is_reported():
-    case = _decode_case([40, 40], 4, 2, 64, seed=5)
+@pytest.mark.parametrize("Hq,Hkv,D", [(4, 2, 64), (16, 4, 128), (16, 8, 64)])
+def test_decode_bad_block_id_is_reported(Hq, Hkv, D):
+    case = _decode_case([40, 40], Hq, Hkv, D, seed=5)
     bt = case.block_tables.clone()
     bt[1, 1] = case.NB + 5                            # outside the pool
     pkv.paged_attention(case.q, case.k_cache, case.v_cache, bt, case.context_lens, case.scale)
@@ -214,12 +215,13 @@ def test_decode_many_short_sequences():
     including empty and one-token contexts."""
     g = torch.Generator().manual_seed(77)
     lens = torch.randint(0, 40, (2100,), generator=g).tolist()
-    case = _decode_case(lens, 8, 2, 64, seed=77)
-    ref = HostCase(case).decode_ref()
-    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
-                              case.scale)
-    assert_close(out, ref, "B=2100")
-    _no_device_error()
+    for Hq, Hkv in ((8, 2), (16, 4)):
+        case = _decode_case(lens, Hq, Hkv, 64, seed=77)
+        ref = HostCase(case).decode_ref()
+        out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                                  case.scale)
+        assert_close(out, ref, f"B=2100 Hq={Hq} Hkv={Hkv}")
+        _no_device_error()
 
 
 def test_decode_ragged_batch_auto_and_split_agree():
