@@ -399,6 +399,8 @@ def extras(peaks, decode_gbs):
     res["llama3_8b_decode_int8"] = {"GB/s": round(gbs, 1), "us": round(ms * 1e3, 2),
                                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "launches": pkv.last_launch_count(),
                                     "bytes": decode_bytes(c), "kv_bytes_vs_bf16": 0.5 + 2.0 / c.D,
+                                    "traffic": profiled_traffic("decode_attn_i8", source_hash(
+                                        "decode_attn_i8.cuh", "decode_attn.cuh", "tcgen05.cuh", "pkv_common.cuh")),
                                     "l2": "inputs larger than L2"}
     T = c.new_key.shape[0]
     nb = 2 * T * c.Hkv * c.D * 2 + 2 * T * c.Hkv * (c.D + 4) + 8 * T
