@@ -18,11 +18,11 @@
 // that integer times k_scale * scale * log2(e) * 2^-e_h.  V stays on the CUDA
 // cores (the probabilities are fp32), exactly as in the CUDA-core kernel.
 //
-// One CTA per (split, head group, sequence), 4 consumer warps and one warp
-// that loads and issues the MMAs.  A tile is 8 pages = 128 keys (the MMA's
+// One CTA per (split, head group, sequence), 4 consumer warps and two loader
+// warps: one loads K and issues the MMAs, one loads V and the row scales.  A tile is 8 pages = 128 keys (the MMA's
 // M): their K codes arrive by tiled TMA into 128- (D=128) or 64-byte (D=64)
 // swizzled rows, their V codes by 1-D bulk copies, their row scales by
-// 16-byte cp.async from the producer warp's lanes.  The MMA
+// 16-byte cp.async from the second loader warp's lanes.  The MMA
 // writes the tile's scores into one of two TMEM buffers (16 columns each);
 // consumer warp w owns TMEM lanes 32w..32w+31, i.e. the tile's keys
 // 32w..32w+31 (pages 2w, 2w+1), and keeps its own online-softmax state over
@@ -43,7 +43,7 @@ struct DecodeI8Shape {
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(HG == 1 || HG == 2 || HG == 4, "heads per CTA");
   static constexpr int NW = 4;                    // consumer warps
-  static constexpr int THREADS = (NW + 1) * 32;   // + the load / MMA warp
+  static constexpr int THREADS = (NW + 2) * 32;   // + a K/MMA warp and a V/scales warp
   static constexpr int TILE_PAGES = 8;
   static constexpr int TILE_ROWS = TILE_PAGES * kPageRows;  // 128 = MMA M
   static constexpr int WROWS = TILE_ROWS / NW;              // 32 keys per consumer warp
@@ -95,7 +95,8 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   const int kvh = hsub / p.nsub;
   const int head0 = kvh * p.G + (hsub % p.nsub) * HG;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool producer = warp == S::NW;
+  const bool producer = warp >= S::NW;  // a loader warp
+  const int lid = warp - S::NW;          // 0: K codes by TMA and the MMAs; 1: V codes and row scales
 
   int L = __ldg(p.context_lens + b);
   const int wp0 = WIN ? window_first_key(L < 0 ? 0 : min(L, p.cap_tokens), p.window) / kPageRows : 0;
@@ -138,10 +139,10 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   float* cq = reinterpret_cast<float*>(sbase + S::MISC_OFF + 16);  // per head: scale * log2(e) * 2^-e_h
 
   // ------------------------------------------------------------- set-up --
-  if (producer) {
+  if (producer && lid == 0) {
     if (lane == 0) {
       for (int s = 0; s < S::ST; ++s) {
-        mbar_init(full(s), 1 + 32);  // the bytes of the bulk copies, then one per lane's row scales
+        mbar_init(full(s), 2 + 32);  // each loader's bytes, then one per lane's row scales
         mbar_init(empty(s), S::NW);
       }
       for (int i = 0; i < 2; ++i) {
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
     __syncwarp();
     tc::alloc(smem_addr(tmem_slot), S::TMEM_COLS);
     tc::relinquish_alloc_permit();
-  } else {
+  } else if (!producer) {
     for (int i = threadIdx.x; i < S::Q_BYTES / 16; i += S::NW * 32)
       reinterpret_cast<uint4*>(sbase + S::Q_OFF)[i] = make_uint4(0, 0, 0, 0);
   }
@@ -228,15 +229,20 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
       }
       const int s = i % S::ST;
       const int np = min(S::TILE_PAGES, n - i * S::TILE_PAGES);
+      // Copies are issued from two warps (K from one, V and the row scales
+      // from the other): one thread's copies go out one after another, and
+      // the tile's 16 page copies from one warp held the kernel back.
       const int blk = __shfl_sync(0xffffffffu, ent_cur, ((i & 3) << 3) + (lane & 7));
-      if (lane == 0) mbar_arrive_expect_tx(full(s), np * 2 * S::PAGE);
+      if (lane == 0) mbar_arrive_expect_tx(full(s), np * S::PAGE);
       __syncwarp();
-      if (lane < np) {
-        const size_t page = (size_t)blk * p.Hkv + kvh;
-        tc::tma_load_4d(base + S::K_OFF + s * S::K_TILE + lane * S::PAGE, &tm_k, 0, 0, kvh, blk, full(s));
-        bulk_g2s_hint(base + S::V_OFF + s * S::K_TILE + lane * S::PAGE, p.v_cache + page * S::PAGE, S::PAGE,
-                      full(s), pol);
+      if (lid == 0) {
+        if (lane < np)
+          tc::tma_load_4d(base + S::K_OFF + s * S::K_TILE + lane * S::PAGE, &tm_k, 0, 0, kvh, blk, full(s));
+        return;
       }
+      if (lane < np)
+        bulk_g2s_hint(base + S::V_OFF + s * S::K_TILE + lane * S::PAGE,
+                      p.v_cache + ((size_t)blk * p.Hkv + kvh) * S::PAGE, S::PAGE, full(s), pol);
       // Row scales, 64 bytes per page and pool: as bulk copies they would
       // double the copies of a tile, and a copy costs about the same whatever
       // its size, so the 32 lanes gather them 16 bytes each instead.
@@ -273,12 +279,15 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
       return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
     };
     for (; issued < S::ST && issued < nt; ++issued) issue(issued);
-    bool ok = mma(0);
-    if (ok) mmas = 1;
+    bool ok = true;
+    if (lid == 0) {
+      ok = mma(0);
+      if (ok) mmas = 1;
+    }
     // MMA i + 1 goes out while the consumers work on tile i; the stage of
     // tile i is refilled once they are done with it.
     for (int i = 0; ok && i < nt; ++i) {
-      if (i + 1 < nt) {
+      if (lid == 0 && i + 1 < nt) {
         ok = mma(i + 1);
         if (!ok) break;
         mmas = i + 2;
@@ -403,8 +412,10 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   tc::fence_before_sync();
   __syncthreads();  // every copy landed and every MMA finished (or was drained)
   if (producer) {
-    tc::fence_after_sync();
-    tc::dealloc(tmem, S::TMEM_COLS);
+    if (lid == 0) {
+      tc::fence_after_sync();
+      tc::dealloc(tmem, S::TMEM_COLS);
+    }
   } else {
     // the running max is the warp's; the sums are per key lane: total them,
     // held once per column of lanes so the row-group merge adds them once
