@@ -238,6 +238,61 @@ class OracleSample:
                 f"{self.orc.num_threads()} threads, {secs:.1f} s")
 
 
+def oracle_by_config():
+    """The oracle on each workload the pages' configs name, on all host threads
+    and (configs 1-3) on one: one pass each (best of 3 for the tiny case), wall
+    clock.  Decode in GB/s of algorithmic bytes (cache write included where the
+    workload has one), prefill in GFLOP/s; the tiny case also in microseconds."""
+    import oracle
+    from paged_kv_cache_477_b200 import workloads as wl
+    from paged_kv_cache_477_b200.workloads import bf16_bits
+    orc = oracle.get()
+    cores = orc.num_threads()
+    res = {"threads": cores}
+
+    def decode_args(c):
+        k, v = bf16_bits(c.k_cache).copy(), bf16_bits(c.v_cache).copy()
+        write = None
+        if c.new_key is not None:
+            write = (bf16_bits(c.new_key), bf16_bits(c.new_value), k, v, c.slot_mapping.numpy())
+        return write, (bf16_bits(c.q), k, v, c.block_tables.numpy(), c.context_lens.numpy(), c.scale)
+
+    def run_decode(write, attn):
+        t0 = time.perf_counter()
+        if write is not None:
+            orc.kv_cache_write(*write)
+        orc.paged_attention(*attn)
+        return time.perf_counter() - t0
+
+    for cfg, name, one_core in (("1", "tiny_decode", True), ("2", "llama32_1b_decode", True),
+                                ("3", WORKLOAD, True), ("4", "ragged_long_decode", False)):
+        c = wl.workload(name, device="cpu")
+        write, attn = decode_args(c)
+        nb = decode_bytes(c) + write_bytes(c)
+        entry = {}
+        for label, threads in (("all_cores", cores), ("one_core", 1)):
+            if label == "one_core" and not one_core:
+                continue
+            orc.set_num_threads(threads)
+            reps = 3 if name == "tiny_decode" else 1
+            t = min(run_decode(write, attn) for _ in range(reps))
+            entry[label] = {"GB/s": round(nb / t / 1e9, 4), "s": round(t, 4)}
+            if name == "tiny_decode":
+                entry[label]["us"] = round(t * 1e6, 1)
+        orc.set_num_threads(cores)
+        res[f"config{cfg}_{name}"] = entry
+        del c, write, attn
+    c = wl.workload("chunked_prefill", device="cpu")
+    k, v = bf16_bits(c.k_cache).copy(), bf16_bits(c.v_cache).copy()
+    t0 = time.perf_counter()
+    orc.kv_cache_write(bf16_bits(c.new_key), bf16_bits(c.new_value), k, v, c.slot_mapping.numpy())
+    orc.paged_attention_prefill(bf16_bits(c.q), c.query_start_loc.numpy(), k, v, c.block_tables.numpy(),
+                                c.context_lens.numpy(), c.scale)
+    t = time.perf_counter() - t0
+    res["config5_chunked_prefill"] = {"all_cores": {"GFLOP/s": round(prefill_flops(c) / t / 1e9, 3), "s": round(t, 2)}}
+    return res
+
+
 def oracle_decode_rate(seconds: float):
     """Oracle decode rate on the host cores, repeated passes over a bounded
     sample for about `seconds`.  Returns (GB/s, cores, sample description)."""
@@ -647,6 +702,7 @@ def main():
                 v1, _, desc1 = oracle_decode_rate(min(4.0, args.cpu_seconds))
                 oracle.get().set_num_threads(cores)
                 line["extras"]["oracle_one_core"] = {"value": round(v1, 4), "unit": "GB/s", "sample": desc1}
+                line["extras"]["oracle_by_config"] = oracle_by_config()
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
