@@ -16,20 +16,20 @@
 // qi = 256 hi + lo.  Rows hi (n = h) and lo (n = HG + h) of the MMA's B
 // operand give the exact integer q.k as 256 S_hi + S_lo in s32; the score is
 // that integer times k_scale * scale * log2(e) * 2^-e_h.  V stays on the CUDA
-// cores (the probabilities are fp32), exactly as in the CUDA-core kernel.
+// cores (the probabilities are fp32).
 //
-// One CTA per (split, head group, sequence), 4 consumer warps and two loader
-// warps: one loads K and issues the MMAs, one loads V and the row scales.  A tile is 8 pages = 128 keys (the MMA's
-// M): their K codes arrive by tiled TMA into 128- (D=128) or 64-byte (D=64)
-// swizzled rows, their V codes by 1-D bulk copies, their row scales by
-// 16-byte cp.async from the second loader warp's lanes.  The MMA
-// writes the tile's scores into one of two TMEM buffers (16 columns each);
-// consumer warp w owns TMEM lanes 32w..32w+31, i.e. the tile's keys
-// 32w..32w+31 (pages 2w, 2w+1), and keeps its own online-softmax state over
-// them, merged across warps at the end as in the CUDA-core kernel.  Each
-// lane first takes its own key's weights (one exp per key and head, V scale
-// folded in); then the warp's lanes, 16 elements of D each, accumulate the
-// 32 rows of V codes with those weights.
+// One CTA per (split, head group, sequence): 4 consumer warps and two loader
+// warps, one loading K and issuing the MMAs, one loading V and the row
+// scales.  A tile is 8 pages = 128 keys (the MMA's M): their K codes arrive
+// by tiled TMA into 128- (D=128) or 64-byte (D=64) swizzled rows, their V
+// codes by 1-D bulk copies, their row scales by 16-byte cp.async from the
+// second loader warp's lanes.  The MMA writes the tile's scores into one of
+// two TMEM buffers (16 columns each); consumer warp w owns TMEM lanes
+// 32w..32w+31, i.e. the tile's keys 32w..32w+31 (pages 2w, 2w+1), and keeps
+// its own online-softmax state over them, merged across warps at the end as
+// in the bf16 decode kernel.  Each lane first takes its own key's weights
+// (one exp per key and head, V scale folded in); then the warp's lanes, 16
+// elements of D each, accumulate the 32 rows of V codes with those weights.
 #pragma once
 #include <cuda.h>
 
