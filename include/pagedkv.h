@@ -307,6 +307,26 @@ pkv_status pkv_paged_attention_prefill_window(
     int32_t bs, float scale, int32_t window, pkv_dtype dtype, pkv_stream_t stream);
 
 /*
+ * paged_attention_int8_window -- pkv_paged_attention_int8 under a sliding
+ * window of `window` keys (>= 1): the query at position L-1 sees keys
+ * L-window .. L-1, as pkv_paged_attention_window does over the bf16 cache
+ * (the inference-lab page's sliding-window cache, section "KV缓存实验与长上下文
+ * 优化", over the Tiny-Infer page's INT8 cache, section "推测性解码与INT8量化").
+ * Same plan and workspace as pkv_paged_attention_window
+ * (pkv_paged_attention_window_workspace_size); errors as
+ * pkv_paged_attention_int8.  Pages wholly before the window are never read.
+ */
+pkv_status pkv_paged_attention_int8_window(void* out, const void* q, const void* k_cache,
+                                           const void* v_cache, const float* k_scale,
+                                           const float* v_scale,
+                                           const int32_t* block_tables, int32_t MB,
+                                           const int32_t* context_lens, int32_t B,
+                                           int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                                           int32_t bs, float scale, int32_t window,
+                                           void* workspace, size_t workspace_bytes,
+                                           pkv_stream_t stream);
+
+/*
  * Shared blocks and copy-on-write.  Sequences that share a prefix (parallel
  * sampling from one prompt) can point their block tables at the same
  * physical blocks and copy a block only when one of them is about to write

@@ -86,6 +86,8 @@ class Oracle:
                                                 _I32, _I32]
         lib.ref_paged_attention_int8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32,
                                                  _I32, _I32, _F32]
+        lib.ref_paged_attention_int8_window.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
+                                                        _I32, _I32, _I32, _F32, _I32]
         lib.ref_paged_attention_window.argtypes = [_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32,
                                                    _I32, _F32, _I32]
         lib.ref_paged_attention_prefill_window.argtypes = [_P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
@@ -146,8 +148,9 @@ class Oracle:
         return self._check(rc, "kv_cache_write_int8", allow_bounds)
 
     def paged_attention_int8(self, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale,
-                             allow_bounds=False) -> np.ndarray:
-        """Decode over the int8 pools: attention over the values code * scale."""
+                             allow_bounds=False, window: int = 0) -> np.ndarray:
+        """Decode over the int8 pools: attention over the values code * scale
+        (window > 0: only the query's last `window` keys)."""
         B, Hq, D = q.shape
         NB, Hkv, bs, _ = k_cache.shape
         assert k_cache.dtype == np.int8 and k_scale.dtype == np.float32
@@ -155,9 +158,12 @@ class Oracle:
         context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
         MB = block_tables.shape[1] if block_tables.ndim == 2 else 0
         out = np.zeros((B, Hq, D), dtype=np.float64)
-        rc = self.lib.ref_paged_attention_int8(_ptr(out), _ptr(np.ascontiguousarray(q)), _ptr(k_cache),
-                                               _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
-                                               MB, _ptr(context_lens), B, Hq, Hkv, D, NB, bs, float(scale))
+        args = (_ptr(out), _ptr(np.ascontiguousarray(q)), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale),
+                _ptr(v_scale), _ptr(block_tables), MB, _ptr(context_lens), B, Hq, Hkv, D, NB, bs, float(scale))
+        if window:
+            rc = self.lib.ref_paged_attention_int8_window(*args, int(window))
+        else:
+            rc = self.lib.ref_paged_attention_int8(*args)
         self._check(rc, "paged_attention_int8", allow_bounds)
         return out
 

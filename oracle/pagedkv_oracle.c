@@ -547,16 +547,19 @@ static void attend_row_int8(double* out, const double* q, int32_t D, double scal
   for (int32_t d = 0; d < D; ++d) out[d] /= l;
 }
 
+static int64_t window_start(int64_t p, int32_t W);
+
 /* Decode over the int8 pool; same gather and grouped-query mapping as
- * ref_paged_attention. */
-int ref_paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cache,
-                             const int8_t* v_cache, const float* k_scale,
-                             const float* v_scale, const int32_t* block_tables,
-                             int32_t MB, const int32_t* context_lens, int32_t B,
-                             int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
-                             int32_t bs, float scale) {
+ * ref_paged_attention.  window > 0: only the keys of the query's sliding
+ * window (see the sliding-window section below) are gathered. */
+static int paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cache,
+                                const int8_t* v_cache, const float* k_scale,
+                                const float* v_scale, const int32_t* block_tables,
+                                int32_t MB, const int32_t* context_lens, int32_t B,
+                                int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                                int32_t bs, float scale, int32_t window) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || MB < 0 ||
-      Hq % Hkv != 0)
+      Hq % Hkv != 0 || window < 0)
     return ORC_INVALID;
   for (int32_t b = 0; b < B; ++b)
     if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)MB * bs)
@@ -565,7 +568,9 @@ int ref_paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cac
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t bh = 0; bh < (int64_t)B * Hq; ++bh) {
     const int32_t b = (int32_t)(bh / Hq), h = (int32_t)(bh % Hq);
-    const int64_t n = context_lens[b];
+    const int64_t L = context_lens[b];
+    const int64_t j0 = (window > 0 && L > 0) ? window_start(L - 1, window) : 0;
+    const int64_t n = L - j0;
     const int32_t g = kv_head_of(h, Hq, Hkv);
     const int8_t** kr = (const int8_t**)malloc(sizeof(void*) * (n + 1));
     const int8_t** vr = (const int8_t**)malloc(sizeof(void*) * (n + 1));
@@ -575,7 +580,7 @@ int ref_paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cac
     double* qd = (double*)malloc(sizeof(double) * D);
     int bad = 0;
     for (int64_t j = 0; j < n; ++j) {
-      const int64_t page = j / bs, row = j % bs;
+      const int64_t page = (j0 + j) / bs, row = (j0 + j) % bs;
       const int32_t blk = block_tables[(int64_t)b * MB + page];
       if (blk < 0 || blk >= NB) {
         bad = 1;
@@ -599,6 +604,28 @@ int ref_paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cac
     free(kr); free(vr); free(ks); free(vs); free(s); free(qd);
   }
   return status;
+}
+
+int ref_paged_attention_int8(double* out, const uint16_t* q, const int8_t* k_cache,
+                             const int8_t* v_cache, const float* k_scale,
+                             const float* v_scale, const int32_t* block_tables,
+                             int32_t MB, const int32_t* context_lens, int32_t B,
+                             int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                             int32_t bs, float scale) {
+  return paged_attention_int8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, MB,
+                              context_lens, B, Hq, Hkv, D, NB, bs, scale, 0);
+}
+
+/* Sliding-window decode over the int8 pool (window >= 1). */
+int ref_paged_attention_int8_window(double* out, const uint16_t* q, const int8_t* k_cache,
+                                    const int8_t* v_cache, const float* k_scale,
+                                    const float* v_scale, const int32_t* block_tables,
+                                    int32_t MB, const int32_t* context_lens, int32_t B,
+                                    int32_t Hq, int32_t Hkv, int32_t D, int32_t NB,
+                                    int32_t bs, float scale, int32_t window) {
+  if (window < 1) return ORC_INVALID;
+  return paged_attention_int8(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, MB,
+                              context_lens, B, Hq, Hkv, D, NB, bs, scale, window);
 }
 
 /* ========================================================================= */

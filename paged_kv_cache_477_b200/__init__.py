@@ -61,6 +61,8 @@ EXPORTS = {
     "pkv_kv_cache_write_int8": ([_P, _P, _I64, _I64, _P, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P], _I32),
     "pkv_paged_attention_int8": ([_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32,
                                   _I32, _P, _SZ, _P], _I32),
+    "pkv_paged_attention_int8_window": ([_P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32,
+                                         _F32, _I32, _P, _SZ, _P], _I32),
     "pkv_paged_attention_window": ([_P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32, _I32, _I32, _I32, _F32,
                                     _I32, _P, _SZ, _I32, _P], _I32),
     "pkv_paged_attention_window_workspace_size": ([_I32, _I32, _I32, _I32, _I32, _I32, _I32], _SZ),
@@ -231,10 +233,7 @@ def kv_cache_write_int8(key, value, k_cache, v_cache, k_scale, v_scale, slot_map
     _check(rc, "kv_cache_write_int8")
 
 
-def paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale: float,
-                         out=None, max_context_len: int = 0, workspace: Optional[torch.Tensor] = None,
-                         stream=None) -> torch.Tensor:
-    """Decode over the int8 cache.  q [B, Hq, D] bf16 -> out [B, Hq, D] bf16."""
+def _int8_common(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, out):
     for t, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
         _contig(_dev(t, name, torch.int8), name)
     for t, name in ((k_scale, "k_scale"), (v_scale, "v_scale")):
@@ -252,6 +251,15 @@ def paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, co
         out = torch.empty_like(q)
     else:
         _contig(_dev(out, "out", torch.bfloat16), "out")
+    return NB, Hkv, bs, D, B, Hq, MB, out
+
+
+def paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale: float,
+                         out=None, max_context_len: int = 0, workspace: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Decode over the int8 cache.  q [B, Hq, D] bf16 -> out [B, Hq, D] bf16."""
+    NB, Hkv, bs, D, B, Hq, MB, out = _int8_common(q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                                                  context_lens, out)
     lib = load_library()
     need = int(lib.pkv_paged_attention_workspace_size(B, Hq, Hkv, D, MB, bs, max_context_len))
     if workspace is None and need > 0:
@@ -263,6 +271,26 @@ def paged_attention_int8(q, k_cache, v_cache, k_scale, v_scale, block_tables, co
                                       context_lens.data_ptr(), B, Hq, Hkv, D, NB, bs, float(scale),
                                       int(max_context_len), ws_ptr, ws_bytes, _stream(stream))
     _check(rc, "paged_attention_int8")
+    return out
+
+
+def paged_attention_int8_window(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, scale: float,
+                                window: int, out=None, workspace: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """Decode over the int8 cache under a sliding window of `window` keys."""
+    NB, Hkv, bs, D, B, Hq, MB, out = _int8_common(q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                                                  context_lens, out)
+    lib = load_library()
+    need = int(lib.pkv_paged_attention_window_workspace_size(B, Hq, Hkv, D, MB, bs, int(window)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    rc = lib.pkv_paged_attention_int8_window(out.data_ptr(), q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                                             k_scale.data_ptr(), v_scale.data_ptr(), block_tables.data_ptr(), MB,
+                                             context_lens.data_ptr(), B, Hq, Hkv, D, NB, bs, float(scale),
+                                             int(window), ws_ptr, ws_bytes, _stream(stream))
+    _check(rc, "paged_attention_int8_window")
     return out
 
 

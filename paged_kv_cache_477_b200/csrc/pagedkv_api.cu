@@ -9,6 +9,7 @@
 #include <new>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include <cuda.h>
@@ -213,10 +214,10 @@ pkv_status launch_decode_any(const pkv::DecodeParams& p, int D, int HG, int B, i
 }
 
 // INT8 cache: Q.K^T on the tensor cores (decode_attn_i8.cuh)
-template <int D, int HG>
+template <int D, int HG, bool WIN>
 struct DecodeI8Kernel {
   using S = pkv::DecodeI8Shape<D, HG>;
-  static constexpr auto fn = pkv::decode_attn_i8_kernel<D, HG, false>;
+  static constexpr auto fn = pkv::decode_attn_i8_kernel<D, HG, WIN>;
   static bool prepare(int dev) {
     static int done[kMaxDevices] = {0};
     static std::mutex mu;
@@ -233,33 +234,38 @@ struct DecodeI8Kernel {
   }
 };
 
-template <int D, int HG>
+template <int D, int HG, bool WIN>
 pkv_status launch_decode_i8_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C, cudaStream_t st) {
-  using K = DecodeI8Kernel<D, HG>;
+  using K = DecodeI8Kernel<D, HG, WIN>;
   if (!K::prepare(current_device())) return PKV_ERR_CUDA;
-  // K codes [NB][Hkv][16][D] bytes: one box is one page of one kv head
+  // K codes [NB][Hkv][16][D] bytes: one box is one page of one kv head.  With
+  // no page to name (MB = 0) every context is empty and no copy is issued.
   CUtensorMap tm;
-  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)pkv::kPageRows, (cuuint64_t)Hkv, (cuuint64_t)p.NB};
-  const cuuint64_t strides[3] = {(cuuint64_t)D, (cuuint64_t)pkv::kPageRows * D,
-                                 (cuuint64_t)Hkv * pkv::kPageRows * D};
-  const cuuint32_t box[4] = {(cuuint32_t)D, (cuuint32_t)pkv::kPageRows, 1, 1};
-  if (!make_tmap(&tm, p.k_cache, 4, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8,
-                 D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
-    return PKV_ERR_CUDA;
+  std::memset(&tm, 0, sizeof tm);
+  if (p.MB > 0) {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)pkv::kPageRows, (cuuint64_t)Hkv, (cuuint64_t)p.NB};
+    const cuuint64_t strides[3] = {(cuuint64_t)D, (cuuint64_t)pkv::kPageRows * D,
+                                   (cuuint64_t)Hkv * pkv::kPageRows * D};
+    const cuuint32_t box[4] = {(cuuint32_t)D, (cuuint32_t)pkv::kPageRows, 1, 1};
+    if (!make_tmap(&tm, p.k_cache, 4, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                   D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
+      return PKV_ERR_CUDA;
+  }
   dim3 grid(C, Hkv * nsub, B);
   K::fn<<<grid, K::S::THREADS, K::S::SMEM_BYTES, st>>>(p, tm);
   return launch_status();
 }
 
+template <bool WIN>
 pkv_status launch_decode_i8(const pkv::DecodeParams& p, int D, int HG, int B, int Hkv, int nsub, int C,
                             cudaStream_t st) {
   if (D == 128)
-    return HG == 4 ? launch_decode_i8_t<128, 4>(p, B, Hkv, nsub, C, st)
-           : HG == 2 ? launch_decode_i8_t<128, 2>(p, B, Hkv, nsub, C, st)
-                     : launch_decode_i8_t<128, 1>(p, B, Hkv, nsub, C, st);
-  return HG == 4 ? launch_decode_i8_t<64, 4>(p, B, Hkv, nsub, C, st)
-         : HG == 2 ? launch_decode_i8_t<64, 2>(p, B, Hkv, nsub, C, st)
-                   : launch_decode_i8_t<64, 1>(p, B, Hkv, nsub, C, st);
+    return HG == 4 ? launch_decode_i8_t<128, 4, WIN>(p, B, Hkv, nsub, C, st)
+           : HG == 2 ? launch_decode_i8_t<128, 2, WIN>(p, B, Hkv, nsub, C, st)
+                     : launch_decode_i8_t<128, 1, WIN>(p, B, Hkv, nsub, C, st);
+  return HG == 4 ? launch_decode_i8_t<64, 4, WIN>(p, B, Hkv, nsub, C, st)
+         : HG == 2 ? launch_decode_i8_t<64, 2, WIN>(p, B, Hkv, nsub, C, st)
+                   : launch_decode_i8_t<64, 1, WIN>(p, B, Hkv, nsub, C, st);
 }
 
 template <int D>
@@ -318,7 +324,8 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
     p.lse_part = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) +
                                           round256(rows * D * sizeof(float)));
   }
-  pkv_status s = k_scale    ? launch_decode_i8(p, D, HG, B, Hkv, nsub, C, st)
+  pkv_status s = k_scale    ? (window > 0 ? launch_decode_i8<true>(p, D, HG, B, Hkv, nsub, C, st)
+                                           : launch_decode_i8<false>(p, D, HG, B, Hkv, nsub, C, st))
                  : window > 0 ? launch_decode_any<true>(p, D, HG, B, Hkv, nsub, C, st)
                               : launch_decode_any<false>(p, D, HG, B, Hkv, nsub, C, st);
   if (s != PKV_OK) return s;
@@ -498,6 +505,31 @@ pkv_status pkv_paged_attention_int8(void* out, const void* q, const void* k_cach
 
 // pages a window of W keys can touch: W keys starting anywhere in a page
 int window_pages(int32_t window) { return (int)(((int64_t)window + pkv::kPageRows - 2) / pkv::kPageRows) + 1; }
+
+pkv_status pkv_paged_attention_int8_window(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                           const float* k_scale, const float* v_scale,
+                                           const int32_t* block_tables, int32_t MB, const int32_t* context_lens,
+                                           int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t NB, int32_t bs,
+                                           float scale, int32_t window, void* workspace, size_t workspace_bytes,
+                                           pkv_stream_t stream) {
+  t_launches = 0;
+  pkv_status s = check_decode_args(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq,
+                                    Hkv, D, NB, bs, PKV_BF16);
+  if (s != PKV_OK || B == 0) return s;
+  if (window < 1) return PKV_ERR_INVALID_ARG;
+  if (MB > 0 && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale)))
+    return PKV_ERR_INVALID_ARG;
+  // the plan of pkv_paged_attention_window: over the pages a window touches
+  const int32_t span = (int32_t)std::min<int64_t>((int64_t)window_pages(window) * bs, (int64_t)MB * bs);
+  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, span);
+  if (pl.num_splits > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned16(workspace)))
+    pl = DecodePlan{1, std::max<int32_t>(MB, 1), 0};  // no room: one CTA per head group
+  if (pl.num_splits == 1) pl.pages_per_split = std::max<int32_t>(MB, 1);
+  static const float kNoScale[4] = {0.f, 0.f, 0.f, 0.f};
+  return run_decode(out, q, k_cache, v_cache, block_tables, MB, context_lens, B, Hq, Hkv, D, NB, scale, pl,
+                    workspace, static_cast<cudaStream_t>(stream), k_scale ? k_scale : kNoScale,
+                    v_scale ? v_scale : kNoScale, window);
+}
 
 pkv_status pkv_paged_attention_window(void* out, const void* q, const void* k_cache, const void* v_cache,
                                       const int32_t* block_tables, int32_t MB, const int32_t* context_lens,

@@ -526,6 +526,49 @@ def pin_window_equals_truncated_context(orc):
     assert np.array_equal(got, ref)
 
 
+def pin_int8_window_brute_force(orc):
+    """INT8 cache under a sliding window: NumPy full-matrix attention over the
+    dequantised last W keys; a window covering the context equals the
+    unwindowed INT8 decode bit for bit."""
+    rng = np.random.default_rng(45)
+    for lens, Hq, Hkv, W in (([5, 17, 1, 33], 4, 2, 7), ([40, 9], 6, 3, 16), ([16], 2, 2, 1)):
+        D, bs = 16, 4
+        k, v, ks, vs, bt, cl = _random_int8_paged(rng, lens, Hkv, D, bs)
+        q = rand_bits(rng, (len(lens), Hq, D))
+        got = orc.paged_attention_int8(q, k, v, ks, vs, bt, cl, 0.3, window=W)
+        kd = k.astype(np.float64) * ks.astype(np.float64)[..., None]
+        vd = v.astype(np.float64) * vs.astype(np.float64)[..., None]
+        G = Hq // Hkv
+        for b, L in enumerate(lens):
+            pages = bt[b, :-(-L // bs)]
+            K = np.transpose(kd[pages], (0, 2, 1, 3)).reshape(-1, Hkv, D)[:L][max(0, L - W):]
+            V = np.transpose(vd[pages], (0, 2, 1, 3)).reshape(-1, Hkv, D)[:L][max(0, L - W):]
+            K, V = np.repeat(K, G, axis=1), np.repeat(V, G, axis=1)
+            S = np.einsum("hd,jhd->hj", bf16_bits_to_f64(q[b]), K) * np.float64(np.float32(0.3))
+            P = np.exp(S - S.max(axis=1, keepdims=True))
+            ref = np.einsum("hj,jhd->hd", P / P.sum(axis=1, keepdims=True), V)
+            assert np.allclose(got[b], ref, rtol=1e-12, atol=1e-14), np.abs(got[b] - ref).max()
+        full = orc.paged_attention_int8(q, k, v, ks, vs, bt, cl, 0.3)
+        assert np.array_equal(orc.paged_attention_int8(q, k, v, ks, vs, bt, cl, 0.3, window=max(lens)), full)
+
+
+def pin_int8_window_equals_bf16_window_on_exact_values(orc):
+    """Power-of-two scales make code * scale bf16-exact: the INT8 window decode
+    then equals the (pinned) bf16 window decode of the same values bit for bit."""
+    rng = np.random.default_rng(46)
+    lens, Hq, Hkv, D, bs = [23, 7, 40], 8, 2, 32, 8
+    k, v, ks, vs, bt, cl = _random_int8_paged(rng, lens, Hkv, D, bs)
+    ks = np.ldexp(1.0, -rng.integers(4, 9, size=ks.shape)).astype(np.float32)
+    vs = np.ldexp(1.0, -rng.integers(4, 9, size=vs.shape)).astype(np.float32)
+    kb = f32_to_bf16_bits(k.astype(np.float32) * ks[..., None])
+    vb = f32_to_bf16_bits(v.astype(np.float32) * vs[..., None])
+    q = rand_bits(rng, (len(lens), Hq, D))
+    for W in (1, 5, 17, 64):
+        a = orc.paged_attention_int8(q, k, v, ks, vs, bt, cl, 0.125, window=W)
+        b = orc.paged_attention_window(q, kb, vb, bt, cl, 0.125, W)
+        assert np.array_equal(a, b), W
+
+
 def pin_window_prefill_brute_force_and_last_row(orc):
     rng = np.random.default_rng(44)
     lens, qlens, Hq, Hkv, D, bs = [40, 9, 25], [12, 9, 1], 4, 2, 16, 4
@@ -647,6 +690,8 @@ ALL_PINS = [
     pin_window_one_returns_last_v,
     pin_window_equals_truncated_context,
     pin_window_prefill_brute_force_and_last_row,
+    pin_int8_window_brute_force,
+    pin_int8_window_equals_bf16_window_on_exact_values,
     pin_rope_position_zero_is_identity,
     pin_rope_unit_vectors_d4,
     pin_rope_keeps_norms_and_relative_position,

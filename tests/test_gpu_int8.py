@@ -170,3 +170,42 @@ def test_int8_decode_bad_block_id_is_reported():
     pkv.paged_attention_int8(case.q, case.k_cache, case.v_cache, case.k_scale, case.v_scale, bt,
                              case.context_lens, case.scale)
     assert pkv.get_device_error() == 5
+
+
+# --------------------------------------------------------------------------- #
+# sliding window over the INT8 cache                                           #
+# --------------------------------------------------------------------------- #
+
+def _decode_window(case, window, **kw):
+    return pkv.paged_attention_int8_window(case.q, case.k_cache, case.v_cache, case.k_scale, case.v_scale,
+                                           case.block_tables, case.context_lens, case.scale, window, **kw)
+
+
+def _window_ref(case, window):
+    h = HostCase(case)
+    return oracle.get().paged_attention_int8(h.q, h.k, h.v, h.ks, h.vs, h.bt, h.lens, case.scale, window=window)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("window", [1, 15, 16, 17, 100, 1000])
+def test_int8_decode_window_edges(D, window):
+    case = _case(EDGE_LENS, 8, 2, D, seed=240 + D + window)
+    out = _decode_window(case, window)
+    assert_close(out, _window_ref(case, window), f"int8 window={window} D={D}")
+    assert torch.count_nonzero(out[0]) == 0
+    assert pkv.get_device_error() == 0
+
+
+@pytest.mark.parametrize("window", [64, 500, 4096])
+def test_int8_decode_window_long_contexts_split(window):
+    """Long contexts: the window plan splits the pages a window touches."""
+    case = _case([5000, 3, 0, 17, 1200, 4096, 640, 33] * 2, 32, 8, 128, seed=250 + window)
+    out = _decode_window(case, window)
+    assert_close(out, _window_ref(case, window), f"int8 window={window} split")
+    assert pkv.get_device_error() == 0
+
+
+def test_int8_decode_window_rejects_zero():
+    case = _case([40], 4, 2, 64, seed=260)
+    with pytest.raises(pkv.PagedKVError):
+        _decode_window(case, 0)
