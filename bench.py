@@ -457,12 +457,40 @@ def extras(peaks, decode_gbs):
                                     "traffic": profiled_traffic("decode_attn_i8", source_hash(
                                         "decode_attn_i8.cuh", "decode_attn.cuh", "tcgen05.cuh", "pkv_common.cuh")),
                                     "l2": "inputs larger than L2"}
+    # the same batch under a 1024-key sliding window
+    W = 1024
+    wsw = torch.empty(max(1, pkv.window_workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, W)), dtype=torch.uint8,
+                      device="cuda")
+    fnw = lambda: pkv.paged_attention_int8_window(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_tables,
+                                                  c.context_lens, c.scale, W, out=out, workspace=wsw)
+    us = timed_us(fnw, 20)
+    wb = sum(min(L, W) for L in c.lens) * c.Hkv * (c.D + 4) * 2 + 2 * c.B * c.Hq * c.D * 2 + \
+        sum(-(-min(L, W) // 16) for L in c.lens) * 4 + c.B * 4
+    res["llama3_8b_decode_int8_window1024"] = {"GB/s": round(wb / (us * 1e-6) / 1e9, 1), "us": round(us, 2),
+                                               "frac_hbm": round(wb / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                                               "launches": pkv.last_launch_count(), "bytes": wb,
+                                               "l2": "window codes of 128 x 8 heads: 268 MiB, larger than L2"}
+    del wsw
     T = c.new_key.shape[0]
     nb = 2 * T * c.Hkv * c.D * 2 + 2 * T * c.Hkv * (c.D + 4) + 8 * T
     us = timed_us(lambda: pkv.kv_cache_write_int8(c.new_key, c.new_value, c.k_cache, c.v_cache, c.k_scale,
                                                   c.v_scale, c.slot_mapping))
     res["kv_cache_write_int8_128"] = {"us": round(us, 2), "GB/s": round(nb / (us * 1e-6) / 1e9, 1), "tokens": T,
                                       "bytes": nb, "l2": "new rows warm in L2; rows scattered into the int8 pool"}
+    del c, out, ws
+    torch.cuda.empty_cache()
+    # INT8 cache at the Llama-3.2-1B shape (D=64)
+    c = wl.workload("llama32_1b_decode", device="cuda", kv_dtype="int8")
+    out = torch.empty_like(c.q)
+    ws = torch.empty(max(1, pkv.workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, 4096)), dtype=torch.uint8,
+                     device="cuda")
+    us = timed_us(lambda: pkv.paged_attention_int8(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_tables,
+                                                   c.context_lens, c.scale, out=out, max_context_len=4096,
+                                                   workspace=ws), 20)
+    res["llama32_1b_decode_int8"] = {"GB/s": round(decode_bytes(c) / (us * 1e-6) / 1e9, 1), "us": round(us, 2),
+                                     "frac_hbm": round(decode_bytes(c) / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                                     "launches": pkv.last_launch_count(), "bytes": decode_bytes(c),
+                                     "l2": "inputs larger than L2"}
     del c, out, ws
     torch.cuda.empty_cache()
     c = wl.workload("chunked_prefill", device="cuda")
