@@ -467,6 +467,7 @@ __global__ void __launch_bounds__(NW * 32)
   // land in it (only possible after a timeout).
   if (done < issued && lane == 0) drain_ring<SW>(wbar, issued);
   __syncwarp();
+  launch_dependents();  // a merge launched after this kernel may be scheduled now
 
   warp_merge<D, HG>(st);
   // after its last page a warp reuses its own ring for its merge data
@@ -497,6 +498,7 @@ struct MergeParams {
 
 template <int D>
 __global__ void __launch_bounds__(D) lse_merge_kernel(const __grid_constant__ MergeParams p) {
+  grid_dependency_wait();  // the split kernel's partials (no-op when launched plainly)
   const int h = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   int L = __ldg(p.context_lens + b);
   L = L < 0 ? 0 : (L > p.cap_tokens ? p.cap_tokens : L);

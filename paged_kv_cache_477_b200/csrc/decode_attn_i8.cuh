@@ -409,6 +409,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   }
 
   // ---------------------------------------------------------- merge --
+  launch_dependents();  // a merge launched after this kernel may be scheduled now
   tc::fence_before_sync();
   __syncthreads();  // every copy landed and every MMA finished (or was drained)
   if (producer) {

@@ -268,9 +268,23 @@ pkv_status launch_decode_i8(const pkv::DecodeParams& p, int D, int HG, int B, in
                    : launch_decode_i8_t<64, 1, WIN>(p, B, Hkv, nsub, C, st);
 }
 
+// The merge is launched as a programmatic dependent of the split kernel: its
+// grid is scheduled while the last split CTAs finish, and each merge CTA
+// waits (griddepcontrol.wait) until the split kernel has completed and its
+// partials are visible, so the launch gap between the two is hidden.
 template <int D>
 pkv_status launch_merge_t(const pkv::MergeParams& mp, int B, int Hq, cudaStream_t st) {
-  pkv::lse_merge_kernel<D><<<dim3(Hq, B), D, 0, st>>>(mp);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(Hq, B);
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pkv::lse_merge_kernel<D>, mp) != cudaSuccess) return PKV_ERR_CUDA;
   return launch_status();
 }
 

@@ -134,6 +134,14 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched after this one with
+// programmatic stream serialization may be scheduled once every CTA here has
+// called launch_dependents (or exited); it calls grid_dependency_wait before
+// touching this kernel's results, which returns once this grid has completed
+// and its memory is visible.  Both are no-ops without such a launch.
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------ numerics ----
 // Hardware base-2 exponential (MUFU.EX2): ex2.approx, flush-to-zero.
 __device__ __forceinline__ float ex2(float x) {
