@@ -516,6 +516,18 @@ def extras(peaks, decode_gbs):
         us = timed_us(fn, 20)
         res["chunked_prefill_warm"] = {"TFLOP/s": round(prefill_flops(c) / (us * 1e-6) / 1e12, 1),
                                        "us": round(us, 2), "l2": "warm (no flush between calls)"}
+        # the same chunks at head size 64 (Llama-3.2-1B's), 32 q / 8 kv heads
+        del c, out
+        c = wl.workload("chunked_prefill", device="cuda", D=64)
+        pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)
+        out = torch.empty_like(c.q)
+        fn = lambda: pkv.paged_attention_prefill(c.q, c.query_start_loc, c.k_cache, c.v_cache, c.block_tables,
+                                                 c.context_lens, c.scale, c.max_q_len, out=out)
+        us = timed_us(fn, 20, flush)
+        tf = prefill_flops(c) / (us * 1e-6) / 1e12
+        res["chunked_prefill_d64"] = {"TFLOP/s": round(tf, 1), "us": round(us, 2),
+                                      "frac_bf16_burst": round(tf / peaks["bf16_tflops"], 4),
+                                      "flops": prefill_flops(c), "l2": "flushed (256 MiB write) before each call"}
     except pkv.PagedKVError as e:
         res["chunked_prefill"] = {"unavailable": str(e)}
     return res

@@ -36,7 +36,7 @@
  *     context length larger than the block table, a wait that ran out) set
  *     the device error word, read with pkv_get_device_error.
  *   - Supported now: dtype PKV_BF16; decode and prefill need bs = 16 and
- *     D in {64, 128} (decode) or D = 128 (prefill); the cache write takes any
+ *     D in {64, 128}; the cache write takes any
  *     bs and any D that is a multiple of 8.  All pointers 16-byte aligned.
  */
 #ifndef PAGEDKV_H
@@ -283,7 +283,7 @@ pkv_status pkv_paged_attention_split_noalloc(
  *   q               : device, [sumQ][Hq][D] bf16
  *   query_start_loc : device, [B+1] int32, query_start_loc[0] = 0
  *   max_q_len       : host upper bound on Q_b (sizes the launch)
- * Needs D = 128, bs = 16, Hq / Hkv dividing 128.
+ * Needs D in {64, 128}, bs = 16, Hq / Hkv dividing 128.
  */
 pkv_status pkv_paged_attention_prefill(
     void* out, const void* q, const int32_t* query_start_loc,

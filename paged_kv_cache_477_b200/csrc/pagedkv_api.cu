@@ -364,15 +364,16 @@ pkv_status run_decode(void* out, const void* q, const void* k_cache, const void*
 }
 
 // ---------------------------------------------------------------- prefill --
+template <int D>
 int prefill_prepare(int dev) {
   static int done[kMaxDevices] = {0};
   static std::mutex mu;
   if (dev < 0 || dev >= kMaxDevices) return -1;
   std::lock_guard<std::mutex> g(mu);
   if (!done[dev]) {
-    for (const void* fn : {reinterpret_cast<const void*>(pkv::prefill_attn_kernel<false>),
-                           reinterpret_cast<const void*>(pkv::prefill_attn_kernel<true>)}) {
-      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pkv::pf::SMEM_BYTES) !=
+    for (const void* fn : {reinterpret_cast<const void*>(pkv::prefill_attn_kernel<D, false>),
+                           reinterpret_cast<const void*>(pkv::prefill_attn_kernel<D, true>)}) {
+      if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, pkv::pf::Layout<D>::SMEM_BYTES) !=
           cudaSuccess)
         return -1;
       // the kernel's setmaxnreg split is sized for exactly this register count
@@ -770,7 +771,7 @@ pkv_status prefill_impl(void* out, const void* q, const int32_t* query_start_loc
     return PKV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
-  if (D != pkv::pf::D || bs != pkv::kPageRows || G > pkv::pf::BM || pkv::pf::BM % G != 0)
+  if ((D != 64 && D != 128) || bs != pkv::kPageRows || G > pkv::pf::BM || pkv::pf::BM % G != 0)
     return PKV_ERR_UNSUPPORTED;
   if (!(scale >= 0.f) || scale == INFINITY) return PKV_ERR_UNSUPPORTED;  // also rejects NaN
   if (B == 0 || sumQ == 0 || max_q_len == 0) return PKV_OK;
@@ -780,7 +781,7 @@ pkv_status prefill_impl(void* out, const void* q, const int32_t* query_start_loc
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache))
     return PKV_ERR_INVALID_ARG;
   const int dev = current_device();
-  const int prep = prefill_prepare(dev);
+  const int prep = D == 128 ? prefill_prepare<128>(dev) : prefill_prepare<64>(dev);
   if (prep == -2) return PKV_ERR_UNSUPPORTED;  // build with an unexpected register count
   if (prep < 0) return PKV_ERR_CUDA;
 
@@ -815,10 +816,18 @@ pkv_status prefill_impl(void* out, const void* q, const int32_t* query_start_loc
   p.window = window;
   dim3 grid(Hkv, B, nct);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (window > 0)
-    pkv::prefill_attn_kernel<true><<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, st>>>(p, tm_q, tm_k, tm_v);
-  else
-    pkv::prefill_attn_kernel<false><<<grid, pkv::pf::THREADS, pkv::pf::SMEM_BYTES, st>>>(p, tm_q, tm_k, tm_v);
+  constexpr int S128 = pkv::pf::Layout<128>::SMEM_BYTES, S64 = pkv::pf::Layout<64>::SMEM_BYTES;
+  if (D == 128) {
+    if (window > 0)
+      pkv::prefill_attn_kernel<128, true><<<grid, pkv::pf::THREADS, S128, st>>>(p, tm_q, tm_k, tm_v);
+    else
+      pkv::prefill_attn_kernel<128, false><<<grid, pkv::pf::THREADS, S128, st>>>(p, tm_q, tm_k, tm_v);
+  } else {
+    if (window > 0)
+      pkv::prefill_attn_kernel<64, true><<<grid, pkv::pf::THREADS, S64, st>>>(p, tm_q, tm_k, tm_v);
+    else
+      pkv::prefill_attn_kernel<64, false><<<grid, pkv::pf::THREADS, S64, st>>>(p, tm_q, tm_k, tm_v);
+  }
   pkv_status s = launch_status();
   if (s == PKV_OK) t_launches = 1;
   return s;

@@ -56,19 +56,13 @@ struct PrefillParams {
 };
 
 namespace pf {
-constexpr int D = 128;
 constexpr int BM = 128;                 // query rows per tile
 constexpr int NQT = 2;                  // query tiles per CTA
 constexpr int BN = 128;                 // keys per tile (8 pages)
 constexpr int KSTAGES = 3;
 constexpr int VSTAGES = 2;
-constexpr int HALF_BYTES = 128 * 128;   // 128 rows x 64 bf16 (one head-dim half)
-constexpr int TILE_BYTES = 2 * HALF_BYTES;
+constexpr int HALF_BYTES = 128 * 128;   // 128 rows x 64 bf16 (one 64-element head-dim half)
 constexpr int PAGE_BOX_BYTES = 16 * 128;  // one page, one half
-constexpr int Q_OFF = 0;
-constexpr int K_OFF = Q_OFF + NQT * TILE_BYTES;
-constexpr int V_OFF = K_OFF + KSTAGES * TILE_BYTES;
-constexpr int BAR_OFF = V_OFF + VSTAGES * TILE_BYTES;
 // barriers
 constexpr int B_Q = 0;
 constexpr int B_KFULL = 1;
@@ -80,8 +74,6 @@ constexpr int B_PFULL = B_SFULL + NQT;       // per query tile, 4 arrivals
 constexpr int B_OREADY = B_PFULL + NQT;      // per query tile
 constexpr int B_MMADONE = B_OREADY + NQT;
 constexpr int NUM_BARS = B_MMADONE + 1;
-constexpr int TMEM_SLOT_OFF = BAR_OFF + NUM_BARS * 8;
-constexpr int SMEM_BYTES = TMEM_SLOT_OFF + 16 + 1024;  // + slack to align the base to 1 KB
 constexpr int THREADS = 384;
 constexpr int TMEM_COLS = 512;
 constexpr int TILE_COLS = 256;  // query tile i: scores at i*256, O at i*256 + 128
@@ -99,6 +91,21 @@ constexpr int REGS_LAUNCH = 168;    // 65536 / 384 rounded down to a multiple of
 constexpr int REGS_LOW = 64;        // load / MMA / allocator warpgroup
 constexpr int REGS_HIGH = 216;      // softmax warpgroups
 static_assert(4 * REGS_LOW + 8 * REGS_HIGH <= 12 * REGS_LAUNCH, "register split must fit the launch");
+
+// Shared-memory layout for head size D: tiles of D/64 swizzled 64-element
+// halves (query tiles, then K stages, then V stages), then the barriers.
+template <int D>
+struct Layout {
+  static_assert(D == 64 || D == 128, "head_dim");
+  static constexpr int NH = D / 64;
+  static constexpr int TILE_BYTES = NH * HALF_BYTES;
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + NQT * TILE_BYTES;
+  static constexpr int V_OFF = K_OFF + KSTAGES * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VSTAGES * TILE_BYTES;
+  static constexpr int TMEM_SLOT_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int SMEM_BYTES = TMEM_SLOT_OFF + 16 + 1024;  // + slack to align the base to 1 KB
+};
 }  // namespace pf
 
 // Three-input maximum (one ALU instruction on sm_100).
@@ -167,10 +174,11 @@ __device__ __forceinline__ PrefillTask prefill_task(const PrefillParams& p, int 
 
 // WIN: sliding window of p.window keys (a separate instantiation, so the
 // plain causal kernel carries none of its per-row bounds).
-template <bool WIN>
+template <int D, bool WIN>
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+  using LY = pf::Layout<D>;
   extern __shared__ __align__(16) unsigned char smem_raw[];  // base aligned to 1 KB by hand below
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -189,7 +197,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
   __syncthreads();
   if (s_flag) return;
 
-  auto bar = [&](int i) { return base + pf::BAR_OFF + 8u * i; };
+  auto bar = [&](int i) { return base + LY::BAR_OFF + 8u * i; };
   if (threadIdx.x == 0) {
     mbar_init(bar(pf::B_Q), 1);
     for (int s = 0; s < pf::KSTAGES; ++s) {
@@ -209,13 +217,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     fence_barrier_init();
   }
   if (warp == 2) {
-    tc::alloc(base + pf::TMEM_SLOT_OFF, pf::TMEM_COLS);
+    tc::alloc(base + LY::TMEM_SLOT_OFF, pf::TMEM_COLS);
     tc::relinquish_alloc_permit();
   }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + pf::TMEM_SLOT_OFF);
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sbase + LY::TMEM_SLOT_OFF);
 
   // Register split (per thread): the load/MMA warpgroup gives up registers to
   // the two softmax warpgroups.  4 x REGS_LOW + 8 x REGS_HIGH <= 12 x
@@ -232,12 +240,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       }
       const PrefillTask k = prefill_task<WIN>(p, t);
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar(pf::B_Q), pf::NQT * pf::TILE_BYTES);
+        mbar_arrive_expect_tx(bar(pf::B_Q), pf::NQT * LY::TILE_BYTES);
         for (int i = 0; i < pf::NQT; ++i) {
-          const uint32_t qd = base + pf::Q_OFF + i * pf::TILE_BYTES;
+          const uint32_t qd = base + LY::Q_OFF + i * LY::TILE_BYTES;
           const int z = k.qs + k.p0 + i * PPT;
-          tc::tma_load_3d(qd, &tm_q, 0, k.kvh * G, z, bar(pf::B_Q));
-          tc::tma_load_3d(qd + pf::HALF_BYTES, &tm_q, 64, k.kvh * G, z, bar(pf::B_Q));
+#pragma unroll
+          for (int h = 0; h < LY::NH; ++h)
+            tc::tma_load_3d(qd + h * pf::HALF_BYTES, &tm_q, 64 * h, k.kvh * G, z, bar(pf::B_Q));
         }
       }
       const int32_t* bt = p.block_tables + (size_t)k.b * p.MB;
@@ -261,26 +270,28 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         const int ks = jl % pf::KSTAGES;
         if (lane == 0) {
           if (jl >= pf::KSTAGES) ok = mbar_wait(bar(pf::B_KEMPTY + ks), ((jl / pf::KSTAGES) - 1) & 1);
-          if (ok) mbar_arrive_expect_tx(bar(pf::B_KFULL + ks), pf::TILE_BYTES);
+          if (ok) mbar_arrive_expect_tx(bar(pf::B_KFULL + ks), LY::TILE_BYTES);
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         if (lane < 8) {
-          const uint32_t kd = base + pf::K_OFF + ks * pf::TILE_BYTES + lane * pf::PAGE_BOX_BYTES;
-          tc::tma_load_4d(kd, &tm_k, 0, 0, k.kvh, blk, bar(pf::B_KFULL + ks));
-          tc::tma_load_4d(kd + pf::HALF_BYTES, &tm_k, 64, 0, k.kvh, blk, bar(pf::B_KFULL + ks));
+          const uint32_t kd = base + LY::K_OFF + ks * LY::TILE_BYTES + lane * pf::PAGE_BOX_BYTES;
+#pragma unroll
+          for (int h = 0; h < LY::NH; ++h)
+            tc::tma_load_4d(kd + h * pf::HALF_BYTES, &tm_k, 64 * h, 0, k.kvh, blk, bar(pf::B_KFULL + ks));
         }
         ++issued_k;
         // V tile j
         const int vs = jl % pf::VSTAGES;
         if (lane == 0) {
           if (jl >= pf::VSTAGES) ok = mbar_wait(bar(pf::B_VEMPTY + vs), ((jl / pf::VSTAGES) - 1) & 1);
-          if (ok) mbar_arrive_expect_tx(bar(pf::B_VFULL + vs), pf::TILE_BYTES);
+          if (ok) mbar_arrive_expect_tx(bar(pf::B_VFULL + vs), LY::TILE_BYTES);
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         if (lane < 8) {
-          const uint32_t vd = base + pf::V_OFF + vs * pf::TILE_BYTES + lane * pf::PAGE_BOX_BYTES;
-          tc::tma_load_4d(vd, &tm_v, 0, 0, k.kvh, blk, bar(pf::B_VFULL + vs));
-          tc::tma_load_4d(vd + pf::HALF_BYTES, &tm_v, 64, 0, k.kvh, blk, bar(pf::B_VFULL + vs));
+          const uint32_t vd = base + LY::V_OFF + vs * LY::TILE_BYTES + lane * pf::PAGE_BOX_BYTES;
+#pragma unroll
+          for (int h = 0; h < LY::NH; ++h)
+            tc::tma_load_4d(vd + h * pf::HALF_BYTES, &tm_v, 64 * h, 0, k.kvh, blk, bar(pf::B_VFULL + vs));
         }
         ++issued_v;
       }
@@ -301,20 +312,20 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       // One thread: it alone waits on the barriers it needs and issues every
       // MMA and commit, so no warp-wide vote sits between two MMA groups.
       constexpr uint32_t IDESC_S = tc::idesc_bf16_f32(pf::BM, pf::BN, false, false);
-      constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(pf::BM, pf::D, false, true);
+      constexpr uint32_t IDESC_PV = tc::idesc_bf16_f32(pf::BM, D, false, true);
       // Descriptors are built once; a K step only moves the start address,
       // whose 14-bit field (address >> 4) cannot carry: shared memory < 256 KB.
-      const uint64_t desc_q = tc::smem_desc_sw128(base + pf::Q_OFF, 16, 1024);
-      const uint64_t desc_k = tc::smem_desc_sw128(base + pf::K_OFF, 16, 1024);
-      const uint64_t desc_v = tc::smem_desc_sw128(base + pf::V_OFF, pf::HALF_BYTES, 1024);
-      constexpr uint32_t TILE16 = pf::TILE_BYTES >> 4;
+      const uint64_t desc_q = tc::smem_desc_sw128(base + LY::Q_OFF, 16, 1024);
+      const uint64_t desc_k = tc::smem_desc_sw128(base + LY::K_OFF, 16, 1024);
+      const uint64_t desc_v = tc::smem_desc_sw128(base + LY::V_OFF, pf::HALF_BYTES, 1024);
+      constexpr uint32_t TILE16 = LY::TILE_BYTES >> 4;
       int tk = 0, tv = 0;  // K and V tiles consumed: ring stage and phase
       auto qk = [&](int i) {  // S_i = Q_i K^T for K tile tk
         const int ks = tk % pf::KSTAGES;
         const uint64_t dq = desc_q + i * TILE16, dk = desc_k + ks * TILE16;
         const uint32_t d_s = tmem + i * pf::TILE_COLS;
 #pragma unroll
-        for (int kk = 0; kk < pf::D / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off16 = ((kk >> 2) * pf::HALF_BYTES + (kk & 3) * 32) >> 4;
           tc::mma_ss(d_s, dq + off16, dk + off16, IDESC_S, kk > 0 ? 1u : 0u);
         }
@@ -330,9 +341,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
           if (tail_rows != 0 && tail_page / 8 == j) {
             // rows past the end of the context hold stale data that a zero
             // probability would not cancel if it were NaN: clear them
-            unsigned char* vp = sbase + pf::V_OFF + vs * pf::TILE_BYTES + (tail_page % 8) * pf::PAGE_BOX_BYTES;
+            unsigned char* vp = sbase + LY::V_OFF + vs * LY::TILE_BYTES + (tail_page % 8) * pf::PAGE_BOX_BYTES;
             const int nvec = (16 - tail_rows) * 8;  // 16-byte vectors per half
-            for (int e = 0; e < 2 * nvec; ++e) {
+            for (int e = 0; e < LY::NH * nvec; ++e) {
               const int half = e / nvec, k = e % nvec;
               *reinterpret_cast<uint4*>(vp + half * pf::HALF_BYTES + tail_rows * 128 + k * 16) =
                   make_uint4(0, 0, 0, 0);
@@ -445,7 +456,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             }
             tc::fence_after_sync();
 #pragma unroll
-            for (int c = 0; c < pf::D; c += 32) {
+            for (int c = 0; c < D; c += 32) {
               uint32_t o[32];
               tc::ld_32x32b_x32(o_addr + c, o);
               tc::wait_ld();
@@ -495,11 +506,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       }
       if (ok && __all_sync(0xffffffffu, mbar_wait(bar(pf::B_OREADY + qt), (k.n - k.j0 - 1) & 1))) {
         tc::fence_after_sync();
-        uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)(k.qs + pos) * p.Hq + k.kvh * G + hh) * pf::D);
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)(k.qs + pos) * p.Hq + k.kvh * G + hh) * D);
         // O / l to global memory
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
 #pragma unroll
-        for (int c = 0; c < pf::D; c += 32) {
+        for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
           tc::ld_32x32b_x32(o_addr + c, o);
           tc::wait_ld();

@@ -36,22 +36,33 @@ def _run(case):
     return out, host
 
 
-def _prefill_case(lens, qlens, Hq, Hkv, seed, extra_blocks=2):
+def _prefill_case(lens, qlens, Hq, Hkv, seed, extra_blocks=2, D=128):
     pages = sum(-(-L // 16) for L in lens)
-    return wl.make_case(kind="prefill", B=len(lens), Hq=Hq, Hkv=Hkv, D=128, bs=16, lens=lens, q_len=qlens,
+    return wl.make_case(kind="prefill", B=len(lens), Hq=Hq, Hkv=Hkv, D=D, bs=16, lens=lens, q_len=qlens,
                         seed=seed, device="cuda", pool_blocks=pages + extra_blocks)
 
 
+@pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("Hq,Hkv", [(8, 2), (32, 8), (4, 4), (16, 8), (16, 2)])
-def test_prefill_small_full(Hq, Hkv):
+def test_prefill_small_full(Hq, Hkv, D):
     # ragged chunks, partial last pages (NaN canaries in the tails), a chunk that
     # is the whole context, single-token chunks, several Q tiles per sequence
     lens = [200, 77, 300, 1, 129, 45]
     qlens = [130, 77, 33, 1, 1, 45]
-    case = _prefill_case(lens, qlens, Hq, Hkv, seed=500 + Hq + Hkv)
+    case = _prefill_case(lens, qlens, Hq, Hkv, seed=500 + Hq + Hkv + D, D=D)
     out, host = _run(case)
     ref, tok = host.prefill_ref()
-    assert_close(out[tok], ref, f"prefill Hq={Hq} Hkv={Hkv}")
+    assert_close(out[tok], ref, f"prefill Hq={Hq} Hkv={Hkv} D={D}")
+    assert pkv.get_device_error() == 0
+
+
+def test_prefill_llama32_1b_shaped_chunks():
+    """Head size 64 at the Llama-3.2-1B shape (32 q / 8 kv heads): 512-token
+    chunks after cached context, every row checked."""
+    case = _prefill_case([1536, 700, 512], [512, 300, 512], 32, 8, seed=620, D=64)
+    out, host = _run(case)
+    ref, tok = host.prefill_ref()
+    assert_close(out[tok], ref, "prefill D=64 Llama-3.2-1B shape")
     assert pkv.get_device_error() == 0
 
 
@@ -118,14 +129,15 @@ def test_prefill_zero_scale_gives_mean_of_visible_values():
     assert pkv.get_device_error() == 0
 
 
+@pytest.mark.parametrize("D", [128, 64])
 @pytest.mark.parametrize("window", [1, 17, 128, 129, 300, 5000])
-def test_prefill_window(window):
+def test_prefill_window(window, D):
     """Sliding window: tiles below every row's window skipped, edge tiles masked
     per row (windows shorter than a tile, tile-aligned, spanning tiles, wider
     than the context)."""
     lens = [700, 77, 1300, 45]
     qlens = [300, 77, 129, 1]
-    case = _prefill_case(lens, qlens, 16, 4, seed=560 + window)
+    case = _prefill_case(lens, qlens, 16, 4, seed=560 + window + D, D=D)
     host = HostCase(case)
     pkv.kv_cache_write(case.new_key, case.new_value, case.k_cache, case.v_cache, case.slot_mapping)
     out = pkv.paged_attention_prefill_window(case.q, case.query_start_loc, case.k_cache, case.v_cache,
