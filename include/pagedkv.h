@@ -167,10 +167,14 @@ pkv_status pkv_kv_cache_write_int8(const void* key, const void* value,
 
 /*
  * paged_attention_int8 -- pkv_paged_attention over the int8 cache: the same
- * plan, launch shapes, workspace (pkv_paged_attention_workspace_size) and
- * errors; K and V are read as codes and scaled by their row's scale inside
- * the kernel (half the bytes of the bf16 cache, plus 4 bytes per row).
- * q and out are bf16 as for pkv_paged_attention; D in {64, 128}, bs = 16.
+ * split plan, workspace (pkv_paged_attention_workspace_size) and errors; K and
+ * V are read as codes and scaled by their row's scale inside the kernel (half
+ * the bytes of the bf16 cache, plus 4 bytes per row).  q and out are bf16 as
+ * for pkv_paged_attention; D in {64, 128}, bs = 16.  The scores q.k are
+ * taken on the tensor cores from the codes directly, with q held per head as
+ * a 15-bit fixed-point pair of signed bytes (exact for every element within
+ * 2^7 of the head's largest magnitude; smaller ones to 2^-14 of it), so the
+ * result differs from attention over code * scale by that rounding of q.
  */
 pkv_status pkv_paged_attention_int8(void* out, const void* q, const void* k_cache,
                                     const void* v_cache, const float* k_scale,

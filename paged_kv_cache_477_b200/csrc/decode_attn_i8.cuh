@@ -64,7 +64,7 @@ struct DecodeI8Shape {
   static constexpr int S_OFF = V_OFF + ST * K_TILE;
   static constexpr int P_OFF = S_OFF + ST * SC_STAGE;       // scores [NW][WROWS][4] fp32
   static constexpr int BAR_OFF = P_OFF + NW * WROWS * 16;   // full[ST] empty[ST] sfull[2] sfree[2]
-  static constexpr int MISC_OFF = BAR_OFF + (2 * ST + 4) * 8;  // tmem base, cq[4], stop flag
+  static constexpr int MISC_OFF = BAR_OFF + (2 * ST + 4) * 8;  // TMEM base address, cq[4]
   static constexpr int SMEM_BYTES = MISC_OFF + 32 + 1024;      // + room to align the base
   // one warp's merge data, in the K ring after the last tile
   static constexpr int MERGE_STRIDE = (HG * D + 2 * HG + 3) / 4 * 4;
@@ -86,16 +86,15 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
     decode_attn_i8_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ CUtensorMap tm_k) {
   using S = DecodeI8Shape<D, HG>;
   extern __shared__ __align__(128) unsigned char smem_i8[];
-  unsigned char* smem_raw = smem_i8;
-  const uint32_t raw_addr = smem_addr(smem_raw);
-  const uint32_t base = (raw_addr + 1023u) & ~1023u;
-  unsigned char* sbase = smem_raw + (base - raw_addr);
+  const uint32_t raw_addr = smem_addr(smem_i8);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;  // swizzled tiles start on 1 KB
+  unsigned char* sbase = smem_i8 + (base - raw_addr);
 
   const int split = blockIdx.x, hsub = blockIdx.y, b = blockIdx.z;
   const int kvh = hsub / p.nsub;
   const int head0 = kvh * p.G + (hsub % p.nsub) * HG;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool producer = warp >= S::NW;  // a loader warp
+  const bool loader = warp >= S::NW;
   const int lid = warp - S::NW;          // 0: K codes by TMA and the MMAs; 1: V codes and row scales
 
   int L = __ldg(p.context_lens + b);
@@ -109,7 +108,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
     return (w < p.pages_per_split && pg0 + w < p.MB) ? __ldg(btrow + pg0 + w) : 0;
   };
   int ent_cur = 0, ent_nxt = 0;
-  if (producer) {
+  if (loader) {
     ent_cur = load_raw(0);
     ent_nxt = load_raw(1);
   }
@@ -139,7 +138,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   float* cq = reinterpret_cast<float*>(sbase + S::MISC_OFF + 16);  // per head: scale * log2(e) * 2^-e_h
 
   // ------------------------------------------------------------- set-up --
-  if (producer && lid == 0) {
+  if (loader && lid == 0) {
     if (lane == 0) {
       for (int s = 0; s < S::ST; ++s) {
         mbar_init(full(s), 2 + 32);  // each loader's bytes, then one per lane's row scales
@@ -154,7 +153,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
     __syncwarp();
     tc::alloc(smem_addr(tmem_slot), S::TMEM_COLS);
     tc::relinquish_alloc_permit();
-  } else if (!producer) {
+  } else if (!loader) {
     for (int i = threadIdx.x; i < S::Q_BYTES / 16; i += S::NW * 32)
       reinterpret_cast<uint4*>(sbase + S::Q_OFF)[i] = make_uint4(0, 0, 0, 0);
   }
@@ -196,7 +195,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
       *reinterpret_cast<uint16_t*>(qs + swizzled_offset<D>(HG + warp, d0)) = (uint16_t)lo;
     }
   }
-  if (!producer) fence_proxy_async_smem();  // the MMA reads the q rows (and zeros) through the async proxy
+  if (!loader) fence_proxy_async_smem();  // the MMA reads the q rows (and zeros) through the async proxy
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -208,7 +207,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   st.reset();
   const int rg = lane / (D / 16), sub = lane % (D / 16);
 
-  if (producer) {
+  if (loader) {
     // ------------------------------------------------- loads and MMAs --
     int chunk = 0;
     auto validate = [&](int e, int c) {  // entries of the CTA's pages must lie in the pool
@@ -412,7 +411,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   launch_dependents();  // a merge launched after this kernel may be scheduled now
   tc::fence_before_sync();
   __syncthreads();  // every copy landed and every MMA finished (or was drained)
-  if (producer) {
+  if (loader) {
     if (lid == 0) {
       tc::fence_after_sync();
       tc::dealloc(tmem, S::TMEM_COLS);
@@ -432,7 +431,7 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
                       2 * sub, 2 * sub + 1);
   }
   __syncthreads();
-  if (producer) return;
+  if (loader) return;
   const size_t row = (size_t)b * p.Hq + head0;
   const float* parts = reinterpret_cast<const float*>(sbase + S::K_OFF);
   if (p.num_splits == 1)
