@@ -44,7 +44,7 @@ def test_binding_covers_every_symbol():
 
 
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         assert lib.pkv_status_string(code)
 
 
@@ -71,6 +71,17 @@ def test_host_validation_needs_no_gpu(lib):
     # workspace sizes are pure host arithmetic
     assert lib.pkv_split_workspace_size(2, 4, 64, 1) == 0
     assert lib.pkv_split_workspace_size(2, 4, 64, 3) == 2 * 4 * 3 * 64 * 4 + 256  # partials + lse
+    # a pool with no blocks cannot back a non-empty block table
+    assert lib.pkv_paged_attention(P, P, P, P, P, 4, P, 1, 4, 2, 64, 0, 16, 1.0, 0, P, 0, 0, P) == 1
+    # the window entry points validate on the host and launch nothing (here: null pointers, window 0)
+    assert lib.pkv_paged_attention_window(P, P, P, P, P, 4, P, 1, 4, 2, 64, 4, 16, 1.0, 0, P, 0, 0, P) == 1
+    assert lib.pkv_paged_attention_int8_window(P, P, P, P, P, P, P, 4, P, 1, 4, 2, 64, 4, 16, 1.0, 0, P, 0,
+                                               P) == 1
+    # prefill: head sizes 64 and 128 only, block size 16 only
+    pf = lambda D, bs: (P, P, P, P, P, P, 4, P, 1, 8, 8, 4, 2, D, 4, bs, 1.0, 0, P)
+    assert lib.pkv_paged_attention_prefill(*pf(96, 16)) == 2
+    assert lib.pkv_paged_attention_prefill(*pf(64, 32)) == 2
+    assert lib.pkv_paged_attention_prefill(*pf(64, 16)) == 1      # null pointers
 
 
 def test_product_path_fails_loudly_without_library(tmp_path):
