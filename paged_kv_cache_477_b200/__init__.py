@@ -20,7 +20,10 @@ Calls (same names as the C ABI):
     paged_attention_window(q, k_cache, v_cache, block_tables, context_lens, scale, window, ...)
     paged_attention_prefill_window(q, query_start_loc, k_cache, v_cache, block_tables,
                                    context_lens, scale, max_q_len, window, ...)
+    paged_attention_int8_window(q, k_cache, v_cache, k_scale, v_scale, block_tables,
+                                context_lens, scale, window, ...)
     copy_blocks(k_cache, v_cache, pairs);  BlockAllocator(num_blocks)
+    hbm_read_probe(buf, sink, chunk_bytes)      (measurement utility)
 """
 from __future__ import annotations
 
