@@ -666,7 +666,8 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     elapsed_ms = t0.elapsed_time(t1)
-    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    attn_each = sorted(a.elapsed_time(b) for a, b in ev)
+    attn_ms = statistics.mean(attn_each)
     clocks = clk.summary()
     attn_launches = pkv.last_launch_count()
     assert pkv.get_device_error() == 0
@@ -756,6 +757,9 @@ def main():
                          "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": peaks["source"],
                          "bytes_per_launch": attn_bytes, "us_per_launch": round(attn_ms * 1e3, 2),
+                         "us_per_launch_spread": {"min": round(attn_each[0] * 1e3, 2),
+                                                  "median": round(statistics.median(attn_each) * 1e3, 2),
+                                                  "max": round(attn_each[-1] * 1e3, 2), "n": len(attn_each)},
                          "traffic": profiled_traffic("decode_attn", src)},
             "e2e": {"value": round(e2e_val, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "how": "pinned host buffers, each step's inputs copied in "

@@ -255,8 +255,16 @@ size_t pkv_split_workspace_size(int32_t B, int32_t Hq, int32_t D,
  *   - A request whose partials need more than PKV_NOALLOC_SCRATCH_BYTES
  *     (pkv_split_workspace_size(B, Hq, D, num_splits)) returns
  *     PKV_ERR_WORKSPACE and launches nothing.
+ *   - The array comes into being when the library's device code is loaded
+ *     on a GPU.  With lazy module loading (the CUDA default) that happens at
+ *     the library's first call on that device, and it costs an allocation and
+ *     a synchronisation there: make any other library call, or one warm-up
+ *     call of this one, first, and the hot path never pays it.
  *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *     that device current) and keeps it for the life of the process; make
+ *     that first call before any stream capture.  Calls after a device reset
+ *     (cudaDeviceReset, or a reset of the primary context) are unsupported:
+ *     the kept address no longer names the array.
  *   - Nothing is allocated or freed by this call, by the library or through
  *     any library routine.
  *   - Every call shares the one array and leaves its partials in it; every

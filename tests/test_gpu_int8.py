@@ -147,9 +147,9 @@ def test_int8_decode_long_contexts_split():
     assert pkv.get_device_error() == 0
 
 
-def test_int8_write_then_decode_llama3_8b_shaped_sampled():
+def test_int8_write_then_decode_llama3_8b_shaped_full():
     """The bench's int8 step: quantise one new token per sequence into the
-    cache, then decode; the written pool is bit-exact, sampled rows in tolerance."""
+    cache, then decode; the written pool is bit-exact, every row in tolerance."""
     case = wl.workload("llama3_8b_decode_int8", device="cuda")
     host = HostCase(case)
     pkv.kv_cache_write_int8(case.new_key, case.new_value, case.k_cache, case.v_cache, case.k_scale,
@@ -158,8 +158,7 @@ def test_int8_write_then_decode_llama3_8b_shaped_sampled():
     host.apply_write()
     assert _same_bits(case.k_cache, host.k) and _same_bits(case.v_cache, host.v)
     assert _same_bits(case.k_scale, host.ks) and _same_bits(case.v_scale, host.vs)
-    rows = [0, 1, 37, 64, 101, 127]
-    assert_close(out[rows], host.decode_ref(rows), "llama3_8b_decode_int8 sampled")
+    assert_close(out, host.decode_ref(), "llama3_8b_decode_int8")
     assert pkv.get_device_error() == 0
 
 

@@ -4,11 +4,9 @@ The chunk's K/V rows are written by the library's cache write first, as a
 caller would; the oracle applies its own cache write to the generator's
 pre-write pool.  Attention outputs must satisfy |gpu - ref| <= 5e-3 + 1e-2 |ref|.
 """
-import numpy as np
 import pytest
 import torch
 
-import oracle
 import paged_kv_cache_477_b200 as pkv
 from paged_kv_cache_477_b200 import workloads as wl
 from parity import HostCase, assert_close
@@ -76,25 +74,15 @@ def test_prefill_empty_chunk_and_long_chunk():
     assert pkv.get_device_error() == 0
 
 
-def test_prefill_workload_sampled_rows():
+def test_prefill_workload_full():
     """The bench's prefill workload (B=4, 512-token chunks after 3584 cached
-    tokens).  Sampled rows: each is checked against decode attention over the
-    keys its position may see, which the oracle's causal pin ties to the
-    chunked definition."""
+    tokens, 32 q / 8 kv heads): every query row of every head against the
+    oracle's chunked causal prefill."""
     case = wl.workload("chunked_prefill", device="cuda")
     out, host = _run(case)
-    qsl = host.qsl
-    rows, qs_rows, lens = [], [], []
-    for b in range(case.B):
-        Q, L = int(qsl[b + 1] - qsl[b]), int(host.lens[b])
-        for i in (0, 1, 31, 32, 127, 128, 255, 300, 510, Q - 1):
-            rows.append(b)
-            qs_rows.append(int(qsl[b]) + i)
-            lens.append(L - Q + i + 1)
-    ref = oracle.get().paged_attention(np.ascontiguousarray(host.q[qs_rows]), host.k, host.v,
-                                       np.ascontiguousarray(host.bt[rows]), np.array(lens, np.int32),
-                                       case.scale)
-    assert_close(out[qs_rows], ref, "chunked_prefill sampled rows")
+    ref, tok = host.prefill_ref()
+    assert len(tok) == case.q.shape[0] == 2048
+    assert_close(out[tok], ref, "chunked_prefill")
     assert pkv.get_device_error() == 0
 
 
