@@ -142,6 +142,8 @@ static double attend_row(double* out, const double* q, int32_t D, double scale,
     for (int32_t d = 0; d < D; ++d) dot += q[d] * bf16_bits_to_f64(kr[d]);
 #if PKV_ORACLE_MUTANT == 3
     s[j] = dot; /* planted: scale dropped */
+#elif PKV_ORACLE_MUTANT == 18
+    s[j] = fabs(scale) * dot; /* planted: sign of the scale dropped */
 #else
     s[j] = scale * dot;
 #endif

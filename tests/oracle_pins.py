@@ -23,6 +23,8 @@ section "分页KV缓存：借鉴操作系统的内存管理"; exact softmax atte
 * GQA equals materialised MHA; G = 1 is plain MHA;
 * split-KV partials merged by log-sum-exp equal the plain result;
 * an empty context gives a zero row;
+* a negative scale: a closed form (weights sigmoid(-2) and sigmoid(2)), the
+  identity (-scale, -q) == (scale, q) bit for bit, and brute force;
 * INT8 cache (one fp32 scale per token row, the reading of the Tiny-Infer
   page's section "推测性解码与INT8量化"): rows built as k * 2^-e decode to
   exactly k and 2^-e; ties round to even; every value is within scale/2 of
@@ -666,6 +668,35 @@ def pin_rope_cache_write(orc):
     assert np.array_equal(k, k0) and np.array_equal(v, v0)   # nothing else touched
 
 
+def pin_negative_scale(orc):
+    """A negative scale is legal attention: the scores scale * q.k reverse
+    their order.  Closed form: keys (1, 0) and (-1, 0), q = (1, 0) and
+    scale -1 give scores -1 and 1, so the weights are sigmoid(-2) and
+    sigmoid(2) (the first query of a two-token chunk sees only key 0).
+    Negating q and the scale together changes nothing, bit for bit, and the
+    NumPy brute force agrees on random chunks."""
+    rng = np.random.default_rng(41)
+    kc = f32_to_bf16_bits(np.array([[1.0, 0.0], [-1.0, 0.0]], np.float32))[None, :, None, :]
+    vc = f32_to_bf16_bits(np.array([[1.0, 0.0], [0.0, 1.0]], np.float32))[None, :, None, :]
+    k, v, bt = scatter_contiguous(orc, kc, vc, [2], 2, rng)
+    q = f32_to_bf16_bits(np.array([[1.0, 0.0], [1.0, 0.0]], np.float32))[:, None, :]
+    lo, hi = 1.0 / (1.0 + np.exp(2.0)), 1.0 / (1.0 + np.exp(-2.0))
+    out = orc.paged_attention_prefill(q, np.array([0, 2], np.int32), k, v, bt, np.array([2], np.int32), -1.0)
+    np.testing.assert_allclose(out[0, 0], [1.0, 0.0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(out[1, 0], [lo, hi], rtol=0, atol=1e-15)
+    dec = orc.paged_attention(q[1:], k, v, bt, np.array([2], np.int32), -1.0)
+    np.testing.assert_allclose(dec[0, 0], [lo, hi], rtol=0, atol=1e-15)
+    for (lens, qlens, Hq, Hkv, D, bs) in [([40, 19], [7, 19], 4, 2, 32, 16), ([9, 33], [9, 5], 6, 2, 16, 4)]:
+        k, v, bt, cl = make_paged(rng, lens, Hkv, D, bs)
+        qsl = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+        q = rand_bits(rng, (int(qsl[-1]), Hq, D))
+        got = orc.paged_attention_prefill(q, qsl, k, v, bt, cl, -0.3)
+        np.testing.assert_allclose(got, brute.paged_attention_prefill(q, qsl, k, v, bt, cl, -0.3), rtol=0,
+                                   atol=1e-12)
+        flipped = orc.paged_attention_prefill(q ^ np.uint16(0x8000), qsl, k, v, bt, cl, 0.3)
+        assert np.array_equal(got, flipped)
+
+
 ALL_PINS = [
     pin_golden_closed_form,
     pin_brute_force_decode,
@@ -696,4 +727,5 @@ ALL_PINS = [
     pin_rope_unit_vectors_d4,
     pin_rope_keeps_norms_and_relative_position,
     pin_rope_cache_write,
+    pin_negative_scale,
 ]

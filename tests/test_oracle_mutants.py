@@ -7,14 +7,15 @@ normaliser dropped, 7 token-major page layout, 8 cache-write slot off by one,
 9 scores taken against V, 10 merge weight sign flipped, 11 int8 code range
 128 instead of 127, 12 int8 rounding toward zero, 13 int8 V rows scaled by the
 K scale, 14 sliding window one key too wide, 15 RoPE pairs adjacent elements,
-16 RoPE turns the wrong way, 17 RoPE frequency exponent halved.
+16 RoPE turns the wrong way, 17 RoPE frequency exponent halved, 18 sign of
+the scale dropped.
 """
 import pytest
 
 import oracle
 import oracle_pins
 
-MUTANTS = list(range(1, 18))
+MUTANTS = list(range(1, 19))
 
 
 @pytest.mark.parametrize("mutant", MUTANTS)
