@@ -773,7 +773,7 @@ pkv_status prefill_impl(void* out, const void* q, const int32_t* query_start_loc
   const int G = Hq / Hkv;
   if ((D != 64 && D != 128) || bs != pkv::kPageRows || G > pkv::pf::BM || pkv::pf::BM % G != 0)
     return PKV_ERR_UNSUPPORTED;
-  if (!(scale >= 0.f) || scale == INFINITY) return PKV_ERR_UNSUPPORTED;  // also rejects NaN
+  if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
   if (B == 0 || sumQ == 0 || max_q_len == 0) return PKV_OK;
   if (!out || !q || !query_start_loc || !k_cache || !v_cache || !block_tables || !context_lens ||
       NB == 0 || MB == 0)
@@ -807,14 +807,14 @@ pkv_status prefill_impl(void* out, const void* q, const int32_t* query_start_loc
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.NB = NB; p.MB = MB; p.G = G; p.sumQ = sumQ;
   p.scale_log2 = scale * 1.4426950408889634f;
   const int ppc = pkv::pf::NQT * (pkv::pf::BM / G);  // query positions per CTA
-  // Query tiles are the slowest grid dimension, launched last tile first: a
-  // later tile sees more keys, so the longest CTAs start in the first wave
-  // and the shortest fill the last one.
+  // Query-tile pairs are the fastest grid dimension, so the CTAs of one
+  // (sequence, kv head) are scheduled together and share its K/V pages
+  // through L2; within a group the last pair (most keys) goes first.
   const int nct = (max_q_len + ppc - 1) / ppc;
-  if (nct > 65535 || B > 65535) return PKV_ERR_UNSUPPORTED;
+  if (Hkv > 65535 || B > 65535) return PKV_ERR_UNSUPPORTED;
   p.nct = nct;
   p.window = window;
-  dim3 grid(Hkv, B, nct);
+  dim3 grid(nct, Hkv, B);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   constexpr int S128 = pkv::pf::Layout<128>::SMEM_BYTES, S64 = pkv::pf::Layout<64>::SMEM_BYTES;
   if (D == 128) {

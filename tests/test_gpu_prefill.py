@@ -99,13 +99,36 @@ def test_prefill_matches_decode_on_last_row():
     assert d <= 2e-2, d
 
 
-def test_prefill_rejects_unsupported_shapes():
+def test_prefill_rejects_unsupported_shapes_and_bad_scales():
     case = _prefill_case([32], [16], 8, 2, seed=602)
+    for scale, status in ((float("nan"), 1), (float("inf"), 1), (float("-inf"), 1)):
+        with pytest.raises(pkv.PagedKVError) as e:
+            pkv.paged_attention_prefill(case.q, case.query_start_loc, case.k_cache, case.v_cache,
+                                        case.block_tables, case.context_lens, scale, case.max_q_len)
+        assert e.value.status == status
+        assert pkv.last_launch_count() == 0
+    odd = _prefill_case([32], [16], 12, 4, seed=604)        # 3 query heads per kv head: 3 does not divide 128
     with pytest.raises(pkv.PagedKVError) as e:
-        pkv.paged_attention_prefill(case.q, case.query_start_loc, case.k_cache, case.v_cache,
-                                    case.block_tables, case.context_lens, -1.0, case.max_q_len)
+        pkv.paged_attention_prefill(odd.q, odd.query_start_loc, odd.k_cache, odd.v_cache, odd.block_tables,
+                                    odd.context_lens, odd.scale, odd.max_q_len)
     assert e.value.status == 2
     assert pkv.last_launch_count() == 0
+
+
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("scale", [-0.125, -1.0])
+def test_prefill_negative_scale(D, scale):
+    """A negative scale reverses the score order (the row maximum of the scaled
+    scores comes from the raw minimum); ragged chunks and partial pages."""
+    lens = [300, 77, 129, 1000]
+    qlens = [130, 77, 1, 257]
+    pages = sum(-(-L // 16) for L in lens)
+    case = wl.make_case(kind="prefill", B=4, Hq=16, Hkv=4, D=D, bs=16, lens=lens, q_len=qlens,
+                        seed=605 + D, device="cuda", pool_blocks=pages + 2, scale=scale)
+    out, host = _run(case)
+    ref, tok = host.prefill_ref()
+    assert_close(out[tok], ref, f"prefill scale={scale} D={D}")
+    assert pkv.get_device_error() == 0
 
 
 def test_prefill_zero_scale_gives_mean_of_visible_values():
