@@ -91,6 +91,23 @@ constexpr int S_COL = 0;                // shared score buffer, 128 columns
 constexpr int P_COL = 128;              // query tile i: P at 128 + 64 i (bf16 pairs)
 constexpr int O_COL = 256;              // query tile i: O at 256 + 128 i
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+// One column pair in poly_every<D>() takes the FMA-pipe exp2 instead of the
+// MUFU one (0: none).  Measured on B200: at head size 64 one pair in eight
+// (507-512 vs 499 TFLOP/s: the exponentials weigh twice as much against MMAs
+// half as long); at 128 none (one in eight: no change, one in four: 1.4 %
+// slower, one in two: 6 % slower).  PKV_PREFILL_POLY_EVERY overrides both.
+template <int D>
+__host__ __device__ constexpr int poly_every() {
+#ifdef PKV_PREFILL_POLY_EVERY
+  return PKV_PREFILL_POLY_EVERY;
+#else
+  return D == 64 ? 8 : 0;
+#endif
+}
+template <int D>
+__host__ __device__ constexpr bool poly_pair(int pair) {
+  return poly_every<D>() > 0 && pair % (poly_every<D>() > 0 ? poly_every<D>() : 1) == poly_every<D>() - 1;
+}
 constexpr int REGS_LAUNCH = 168;    // 65536 / 384 rounded down to a multiple of 8
 // setmaxnreg takes one count per warpgroup: every warp of a warpgroup must
 // execute the same instruction with the same count
@@ -127,8 +144,45 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return r;
 }
 
+// 2^x on the FMA pipe (Cody-Waite style): x = n + f with n = round(x) found by
+// the 1.5 * 2^23 shifter, f in [-0.5, 0.5]; 2^f by a degree-3 polynomial
+// fitted here for minimum relative error on that interval (max relative error
+// 7.5e-5 in fp32, below bf16's 2^-9 rounding of P); n is added to the
+// exponent field.  Inputs are clamped at -126 so n never underflows the
+// exponent; callers zero masked entries themselves.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+  const float2 shifter = make_float2(12582912.f, 12582912.f);
+  const float2 j = __fadd2_rn(x, shifter);            // low mantissa bits hold round(x)
+  const float2 n = __fadd2_rn(j, make_float2(-shifter.x, -shifter.y));  // round(x), exact
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 p = __ffma2_rn(make_float2(0.05517098f, 0.05517098f), f, make_float2(0.24260971f, 0.24260971f));
+  p = __ffma2_rn(p, f, make_float2(0.69326097f, 0.69326097f));
+  p = __ffma2_rn(p, f, make_float2(0.99992818f, 0.99992818f));
+  const uint32_t ex = __float_as_uint(j.x) << 23, ey = __float_as_uint(j.y) << 23;
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + ex), __uint_as_float(__float_as_uint(p.y) + ey));
+}
+
+// One level of a tree of three-input extrema over the first W values of v,
+// then the next level (constant trip counts, so v stays in registers).
+template <bool MAX, int W>
+__device__ __forceinline__ void fold3(float* v) {
+  if constexpr (W > 1) {
+    constexpr int NW = (W + 2) / 3;
+#pragma unroll
+    for (int k = 0; k < NW; ++k) {
+      const float a = v[3 * k];
+      const float b = 3 * k + 1 < W ? v[3 * k + 1] : a;
+      const float c = 3 * k + 2 < W ? v[3 * k + 2] : a;
+      v[k] = MAX ? fmax3(a, b, c) : fmin3(a, b, c);
+    }
+    fold3<MAX, NW>(v);
+  }
+}
+
 // Largest (MAX) or smallest value of N scores: N/16 independent chains of
-// three-input extrema.
+// three-input extrema, folded three at a time.  (A full tree of depth log3 N
+// measured no faster on B200.)
 template <bool MAX, int N>
 __device__ __forceinline__ float row_extreme(const uint32_t* sr) {
   auto e3 = [](float a, float b, float c) { return MAX ? fmax3(a, b, c) : fmin3(a, b, c); };
@@ -142,16 +196,7 @@ __device__ __forceinline__ float row_extreme(const uint32_t* sr) {
     for (int e = 3; e < 15; e += 2) m = e3(m, __uint_as_float(sr[16 * k + e]), __uint_as_float(sr[16 * k + e + 1]));
     ch[k] = e2(m, __uint_as_float(sr[16 * k + 15]));
   }
-#pragma unroll
-  for (int w = NC; w > 1; w = (w + 2) / 3) {  // fold the chains three at a time
-#pragma unroll
-    for (int k = 0; k < (w + 2) / 3; ++k) {
-      const float a = ch[3 * k];
-      const float b = 3 * k + 1 < w ? ch[3 * k + 1] : a;
-      const float c = 3 * k + 2 < w ? ch[3 * k + 2] : a;
-      ch[k] = e3(a, b, c);
-    }
-  }
+  fold3<MAX, NC>(ch);
   return ch[0];
 }
 
@@ -498,8 +543,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         for (int c = 0; c < pf::BN; c += 2) {
           const float2 x =
               __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2x2, negm);
-          float2 pr = make_float2(ex2(x.x), ex2(x.y));
-          if (diag) {  // masked keys: exactly 0 (a zero scale would not give it)
+          float2 pr = pf::poly_pair<D>(c / 2) ? exp2_poly2(x) : make_float2(ex2(x.x), ex2(x.y));
+          if (diag) {  // masked keys: exactly 0 (the polynomial, or a zero scale, would not give it)
             if (kv0 + c > limit || (WIN && kv0 + c < lo)) pr.x = 0.f;
             if (kv0 + c + 1 > limit || (WIN && kv0 + c + 1 < lo)) pr.y = 0.f;
           }
