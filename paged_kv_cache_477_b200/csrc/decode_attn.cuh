@@ -13,12 +13,15 @@
 //   * Work is cut into segments: (sequence b, a group of HG query heads that
 //     share one kv head).  The HG query rows live in registers, so every K/V
 //     byte is read from HBM once per group (grouped-query reuse).
-//   * Every warp feeds itself: lane 0 issues 1-D bulk copies (cp.async.bulk)
-//     of whole pages -- a (block, kv head) page is one contiguous 4 KB (D=128)
-//     or 2 KB (D=64) run -- into the warp's own SW-stage shared-memory ring,
-//     completion tracked by one mbarrier per stage.  A warp refills a stage
-//     as soon as it has read it, so no cross-warp hand-off is needed and no
-//     warp is spent on copies.
+//   * Pages move by 1-D bulk copies (cp.async.bulk) of whole pages -- a
+//     (block, kv head) page is one contiguous 4 KB (D=128) or 2 KB (D=64) run
+//     -- into each warp's own SW-stage shared-memory ring, completion tracked
+//     by one mbarrier per stage.  At D=128 every warp feeds itself: lane 0
+//     refills a stage as soon as the warp has read it.  At D=64 (twice the
+//     copies per byte) each consumer warp has a producer warp that issues its
+//     copies and refills a stage when the consumer hands it back, so copy
+//     issue never interrupts the arithmetic; a register split (setmaxnreg)
+//     keeps two such CTAs per SM.
 //   * Two CTAs per SM (shared-memory carveout at its maximum) keep
 //     2 x NW x SW pages -- about 192 KB -- in flight per SM, which is what
 //     Little's law asks for at full HBM bandwidth.
@@ -73,7 +76,9 @@ __device__ __forceinline__ int window_first_key(int L, int window) {
 
 // A ring stage holds PPS consecutive pages of one sequence: their K pages
 // side by side (ROWS = 16 * PPS contiguous key rows), then their V pages.
-template <int D, int HG, int NW, int SW, int PPS>
+// PROD: each of the NW consumer warps has a producer warp that issues its
+// copies (NW more warps, and an "empty" barrier per stage).
+template <int D, int HG, int NW, int SW, int PPS, bool PROD = false>
 struct DecodeShape {
   static_assert(D == 64 || D == 128, "head_dim");
   static constexpr int LPR = D / 16;              // lanes sharing one key row
@@ -82,15 +87,22 @@ struct DecodeShape {
   static constexpr int TPL = ROWS / RPW;          // rows per lane per stage
   static constexpr int PAGE_BYTES = kPageRows * D * 2;
   static constexpr int STAGE_BYTES = 2 * PPS * PAGE_BYTES;
-  static constexpr int THREADS = NW * 32;
+  static constexpr int THREADS = NW * 32 * (PROD ? 2 : 1);
+  // register split of the producer form: consumers (warpgroup 0) up to
+  // REGS_CONS, producers (warpgroup 1) down to REGS_PROD, within the 128 per
+  // thread that two CTAs of THREADS threads leave each on an SM
+  static constexpr int REGS_CONS = 216, REGS_PROD = 40, REGS_LAUNCH = 128;
+  static_assert(!PROD || (NW == 4 && REGS_CONS + REGS_PROD <= 2 * REGS_LAUNCH), "producer register split");
   static constexpr int WARP_RING = SW * STAGE_BYTES;
   static constexpr int RING_BYTES = NW * WARP_RING;
   // one warp's merge data: acc [HG][D], m [HG], l [HG]; stride kept 16-byte aligned
   static constexpr int MERGE_STRIDE = (HG * D + 2 * HG + 3) / 4 * 4;
   static_assert(MERGE_STRIDE * 4 <= WARP_RING, "merge data must fit the warp's ring");
-  // rings, then barriers (merge data reuses each warp's ring)
+  // rings, then "full" barriers, then (PROD) "empty" barriers; merge data
+  // reuses each warp's ring
   static constexpr int BAR_OFFSET = RING_BYTES;
-  static constexpr int SMEM_BYTES = BAR_OFFSET + NW * SW * 8;
+  static constexpr int EMPTY_OFFSET = BAR_OFFSET + NW * SW * 8;
+  static constexpr int SMEM_BYTES = EMPTY_OFFSET + (PROD ? NW * SW * 8 : 0);
 };
 
 __device__ __forceinline__ float2 widen2(uint32_t w) {
@@ -313,17 +325,22 @@ __device__ __forceinline__ void drain_ring(uint32_t wbar, int issued) {
 
 // ============================================================================
 // One CTA per (split, head group, sequence).
+// PROD: warps NW..2NW-1 are producers; producer warp NW + w issues the copies
+// of consumer warp w's unit stream into w's ring, so the consumers never stop
+// computing to issue copies.
 // ============================================================================
-template <int D, int HG, int NW, int SW, int PPS, bool WIN = false>
-__global__ void __launch_bounds__(NW * 32)
+template <int D, int HG, int NW, int SW, int PPS, bool WIN = false, bool PROD = false>
+__global__ void __launch_bounds__(NW * 32 * (PROD ? 2 : 1), PROD ? 2 : 1)
     decode_attn_kernel(const __grid_constant__ DecodeParams p) {
-  using S = DecodeShape<D, HG, NW, SW, PPS>;
+  using S = DecodeShape<D, HG, NW, SW, PPS, PROD>;
   extern __shared__ __align__(128) unsigned char smem[];
 
   const int split = blockIdx.x, hsub = blockIdx.y, b = blockIdx.z;
   const int kvh = hsub / p.nsub;
   const int head0 = kvh * p.G + (hsub % p.nsub) * HG;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool producer = PROD && warp >= NW;
+  const int cw = warp % NW;  // the consumer warp whose unit stream this warp reads or fills
 
   int L = __ldg(p.context_lens + b);
   // The sequence's pages from the first one its sliding window reaches (WIN;
@@ -331,7 +348,7 @@ __global__ void __launch_bounds__(NW * 32)
   const int wp0 = WIN ? window_first_key(L < 0 ? 0 : min(L, p.cap_tokens), p.window) / kPageRows : 0;
   const int pg0 = wp0 + split * p.pages_per_split;
   // The CTA's pages are cut into units of PPS consecutive pages, one unit per
-  // ring stage; unit j of this warp is unit u = warp + j * NW, pages
+  // ring stage; unit j of consumer warp cw is unit u = cw + j * NW, pages
   // pg0 + u * PPS + i.  Lane l of a chunk holds the block-table entries of
   // unit j = 32 * chunk + l.  The first two chunks are loaded together with
   // the context length (bounded by the table row and the split, not by the
@@ -341,12 +358,13 @@ __global__ void __launch_bounds__(NW * 32)
   struct Entries {
     int blk[PPS];
   };
+  const bool issuer = PROD ? producer : true;  // this warp issues copies
   auto load_raw = [&](int c) {
     Entries e;
 #pragma unroll
     for (int i = 0; i < PPS; ++i) {
-      const int w = (warp + (c * 32 + lane) * NW) * PPS + i;  // page index within the split
-      e.blk[i] = (w < p.pages_per_split && pg0 + w < p.MB) ? __ldg(btrow + pg0 + w) : 0;
+      const int w = (cw + (c * 32 + lane) * NW) * PPS + i;  // page index within the split
+      e.blk[i] = (issuer && w < p.pages_per_split && pg0 + w < p.MB) ? __ldg(btrow + pg0 + w) : 0;
     }
     return e;
   };
@@ -375,22 +393,29 @@ __global__ void __launch_bounds__(NW * 32)
   }
 
   // ------------------------------------------------ this warp's unit stream --
-  const int nu = (n + PPS - 1) / PPS;                           // units of this CTA
-  const int my_n = warp < nu ? (nu - warp + NW - 1) / NW : 0;  // units warp, warp+NW, ...
-  const uint32_t wring = smem_addr(smem) + warp * S::WARP_RING;
-  const uint32_t wbar = smem_addr(smem) + S::BAR_OFFSET + warp * SW * 8;
-  unsigned char* wring_ptr = smem + warp * S::WARP_RING;
-  if (lane == 0) {
-    for (int s = 0; s < SW; ++s) mbar_init(wbar + 8 * s, 1);
+  const int nu = (n + PPS - 1) / PPS;                        // units of this CTA
+  const int my_n = cw < nu ? (nu - cw + NW - 1) / NW : 0;   // units cw, cw+NW, ...
+  const uint32_t wring = smem_addr(smem) + cw * S::WARP_RING;
+  const uint32_t wbar = smem_addr(smem) + S::BAR_OFFSET + cw * SW * 8;    // stage full
+  const uint32_t ebar = smem_addr(smem) + S::EMPTY_OFFSET + cw * SW * 8;  // stage read (PROD)
+  unsigned char* wring_ptr = smem + cw * S::WARP_RING;
+  if (!producer && lane == 0) {
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(wbar + 8 * s, 1);
+      if (PROD) mbar_init(ebar + 8 * s, 1);
+    }
     fence_barrier_init();
   }
-  __syncwarp();
+  if (PROD)
+    __syncthreads();  // the producer uses the barriers its consumer initialised
+  else
+    __syncwarp();
 
   auto validate = [&](Entries e, int c) {  // entries of pages this warp reads must lie in the pool
     const int j = c * 32 + lane;
 #pragma unroll
     for (int i = 0; i < PPS; ++i)
-      if (j < my_n && (warp + j * NW) * PPS + i < n && (e.blk[i] < 0 || e.blk[i] >= p.NB)) {
+      if (j < my_n && (cw + j * NW) * PPS + i < n && (e.blk[i] < 0 || e.blk[i] >= p.NB)) {
         set_error(PKV_ERR_BOUNDS);
         e.blk[i] = 0;  // keep every copy inside the pool
       }
@@ -407,7 +432,7 @@ __global__ void __launch_bounds__(NW * 32)
       bt_cur = validate(bt_nxt, chunk);
       bt_nxt = load_raw(chunk + 1);
     }
-    const int np = min(PPS, n - (warp + k * NW) * PPS);  // pages of this unit (>= 1)
+    const int np = min(PPS, n - (cw + k * NW) * PPS);  // pages of this unit (>= 1)
     int blk[PPS];
 #pragma unroll
     for (int i = 0; i < PPS; ++i) blk[i] = __shfl_sync(0xffffffffu, bt_cur.blk[i], k & 31);
@@ -425,54 +450,87 @@ __global__ void __launch_bounds__(NW * 32)
     }
     ++issued;
   };
-  for (int k = 0; k < SW && k < my_n; ++k) issue_next();
 
-  // ---------------------------------------------------------- registers --
-  const int rg = lane / S::LPR, sub = lane % S::LPR;
-  // bf16: the lane's two 16-byte vectors of a row (D=64 odd row groups in
-  // swapped order); int8: its 16 consecutive elements, i.e. bf16 vectors
-  // 2 * sub and 2 * sub + 1 of q and of the output
-  const int swap = D == 64 ? (rg & 1) : 0;
-  const int ch0 = sub + S::LPR * swap;        // 16-byte vector held in slot 0
-  const int ch1 = sub + S::LPR * (swap ^ 1);  // and in slot 1
-  float2 q2[HG][8];
-  load_q<D, HG>(q2, p.q + ((size_t)b * p.Hq + head0) * D, ch0, ch1, p.scale_log2);
-  LaneState<HG> st;
-  st.reset();
-
-  // valid rows counted from this CTA's first page: the sequence's, and no
-  // further than the CTA's own pages
-  const int rows_cta = min(L - pg0 * kPageRows, n * kPageRows);
-  // rows before the window, counted the same way (<= 0 past the first split)
-  const int lo_cta = WIN ? window_first_key(L, p.window) - pg0 * kPageRows : 0;
-  int done = 0;
-  for (int j = 0; j < my_n; ++j, ++done) {
-    const int s = j % SW;
-    // every lane waits (each needs the acquire); a timeout on any lane stops
-    // the whole warp, which still drains its copies and joins the merge
-    const bool ok = mbar_wait(wbar + 8 * s, (j / SW) & 1);
-    if (!__all_sync(0xffffffffu, ok)) break;
-    const unsigned char* kp = wring_ptr + s * S::STAGE_BYTES;
-    attend_rows<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES, lo_cta - (warp + j * NW) * S::ROWS,
-                                rows_cta - (warp + j * NW) * S::ROWS, rg, ch0, ch1);
-    if (issued < my_n) {
-      // the stage just read is refilled: order the generic-proxy reads of all
-      // lanes before the copy engine's writes
-      fence_proxy_async_smem();
-      __syncwarp();
+  if (producer) {
+    // ------------------------------------------------------------ producer --
+    // Fill the consumer's ring in unit order; a stage is refilled once the
+    // consumer has read it.  Then wait for the last copy into every stage.
+    // (setmaxnreg takes one count per warpgroup: the producers are warpgroup
+    // 1, the consumers warpgroup 0.)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(S::REGS_PROD));
+    for (int k = 0; k < my_n; ++k) {
+      if (k >= SW && !__all_sync(0xffffffffu, mbar_wait(ebar + 8 * (k % SW), ((k / SW) - 1) & 1))) break;
       issue_next();
     }
-  }
-  // Never reuse or leave the ring while one of this warp's copies may still
-  // land in it (only possible after a timeout).
-  if (done < issued && lane == 0) drain_ring<SW>(wbar, issued);
-  __syncwarp();
-  launch_dependents();  // a merge launched after this kernel may be scheduled now
+    if (lane == 0) drain_ring<SW>(wbar, issued);
+    __syncwarp();
+    launch_dependents();
+  } else {
+    if (PROD)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(S::REGS_CONS));
+    else
+      for (int k = 0; k < SW && k < my_n; ++k) issue_next();
 
-  warp_merge<D, HG>(st);
-  // after its last page a warp reuses its own ring for its merge data
-  warp_store<D, HG>(reinterpret_cast<float*>(wring_ptr), st, rg, sub, ch0, ch1);
+    // -------------------------------------------------------- registers --
+    const int rg = lane / S::LPR, sub = lane % S::LPR;
+    // bf16: the lane's two 16-byte vectors of a row (D=64 odd row groups in
+    // swapped order)
+    const int swap = D == 64 ? (rg & 1) : 0;
+    const int ch0 = sub + S::LPR * swap;        // 16-byte vector held in slot 0
+    const int ch1 = sub + S::LPR * (swap ^ 1);  // and in slot 1
+    float2 q2[HG][8];
+    load_q<D, HG>(q2, p.q + ((size_t)b * p.Hq + head0) * D, ch0, ch1, p.scale_log2);
+    LaneState<HG> st;
+    st.reset();
+
+    // valid rows counted from this CTA's first page: the sequence's, and no
+    // further than the CTA's own pages
+    const int rows_cta = min(L - pg0 * kPageRows, n * kPageRows);
+    // rows before the window, counted the same way (<= 0 past the first split)
+    const int lo_cta = WIN ? window_first_key(L, p.window) - pg0 * kPageRows : 0;
+    int done = 0;
+    for (int j = 0; j < my_n; ++j, ++done) {
+      const int s = j % SW;
+      // every lane waits (each needs the acquire); a timeout on any lane stops
+      // the whole warp, which still drains its copies and joins the merge
+      const bool ok = mbar_wait(wbar + 8 * s, (j / SW) & 1);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const unsigned char* kp = wring_ptr + s * S::STAGE_BYTES;
+      attend_rows<D, HG, S::ROWS>(st, q2, kp, kp + PPS * S::PAGE_BYTES, lo_cta - (cw + j * NW) * S::ROWS,
+                                  rows_cta - (cw + j * NW) * S::ROWS, rg, ch0, ch1);
+      if (PROD) {
+        if (j + SW < my_n) {
+          // hand the stage back to the producer: order the generic-proxy reads
+          // of all lanes before the copy engine's writes
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(ebar + 8 * s);
+        }
+      } else if (issued < my_n) {
+        // the stage just read is refilled: order the generic-proxy reads of all
+        // lanes before the copy engine's writes
+        fence_proxy_async_smem();
+        __syncwarp();
+        issue_next();
+      }
+    }
+    // Never reuse or leave the ring while one of this warp's copies may still
+    // land in it (only possible after a timeout).
+    if (!PROD && done < issued && lane == 0) drain_ring<SW>(wbar, issued);
+    __syncwarp();
+    launch_dependents();  // a merge launched after this kernel may be scheduled now
+
+    warp_merge<D, HG>(st);
+    if (PROD && done < my_n) {
+      // a wait ran out: the producer may still be draining copies into this
+      // ring, so the merge data go nowhere (the error word reports the call)
+    } else {
+      // after its last page a warp reuses its own ring for its merge data
+      warp_store<D, HG>(reinterpret_cast<float*>(wring_ptr), st, rg, sub, ch0, ch1);
+    }
+  }
   __syncthreads();
+  if (producer) return;
   const size_t row = (size_t)b * p.Hq + head0;
   const float* parts = reinterpret_cast<const float*>(smem);
   if (p.num_splits == 1)

@@ -97,12 +97,16 @@ constexpr int pages_per_stage(int D) { return D == 128 ? 1 : 2; }
 // stages per warp: 96 KB of pages in flight per CTA, two CTAs per SM
 constexpr int kDecodeStages = 3;
 
+// D=64 pages are 2 KB: twice the copies per byte, issued by producer warps
+constexpr bool decode_producers(int D) { return D == 64; }
+
 template <int D, int HG>
-using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D)>;
+using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D), decode_producers(D)>;
 
 template <int D, int HG, bool WIN = false>
 struct DecodeKernel {
-  static constexpr auto fn = pkv::decode_attn_kernel<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D), WIN>;
+  static constexpr auto fn =
+      pkv::decode_attn_kernel<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D), WIN, decode_producers(D)>;
   // set the dynamic shared-memory limit once per device; return CTAs per SM
   static int prepare(int dev) {
     static int occ[kMaxDevices] = {0};
@@ -115,6 +119,13 @@ struct DecodeKernel {
           cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return -1;
+      if (decode_producers(D)) {
+        // the producer form's setmaxnreg split is sized for exactly this
+        // register count at launch; any other would leave it waiting forever
+        cudaFuncAttributes attr;
+        if (cudaFuncGetAttributes(&attr, fn) != cudaSuccess || attr.numRegs != DecodeS<D, HG>::REGS_LAUNCH)
+          return -2;
+      }
       int n = 0;
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, DecodeS<D, HG>::THREADS,
                                                         DecodeS<D, HG>::SMEM_BYTES) != cudaSuccess ||
@@ -195,7 +206,9 @@ DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, 
 template <int D, int HG, bool WIN = false>
 pkv_status launch_decode_t(const pkv::DecodeParams& p, int B, int Hkv, int nsub, int C, cudaStream_t st) {
   using K = DecodeKernel<D, HG, WIN>;
-  if (K::prepare(current_device()) < 0) return PKV_ERR_CUDA;
+  const int occ = K::prepare(current_device());
+  if (occ == -2) return PKV_ERR_UNSUPPORTED;  // a build whose register count the split does not fit
+  if (occ < 0) return PKV_ERR_CUDA;
   dim3 grid(C, Hkv * nsub, B);
   K::fn<<<grid, DecodeS<D, HG>::THREADS, DecodeS<D, HG>::SMEM_BYTES, st>>>(p);
   return launch_status();
