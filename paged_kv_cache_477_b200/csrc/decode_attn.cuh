@@ -16,14 +16,14 @@
 //   * Pages move by 1-D bulk copies (cp.async.bulk) of whole pages -- a
 //     (block, kv head) page is one contiguous 4 KB (D=128) or 2 KB (D=64) run
 //     -- into each warp's own SW-stage shared-memory ring, completion tracked
-//     by one mbarrier per stage.  At D=128 every warp feeds itself: lane 0
-//     refills a stage as soon as the warp has read it.  At D=64 (twice the
-//     copies per byte) each consumer warp has a producer warp that issues its
-//     copies and refills a stage when the consumer hands it back, so copy
-//     issue never interrupts the arithmetic; a register split (setmaxnreg)
-//     keeps two such CTAs per SM.
+//     by one mbarrier per stage.  Each consumer warp has a producer warp
+//     that issues its copies and refills a stage when the consumer hands it
+//     back, so copy issue never interrupts the arithmetic (it matters most at
+//     D=64, with twice the copies per byte); a register split (setmaxnreg)
+//     keeps two such CTAs per SM.  (Without producers -- PROD = false -- each
+//     warp's lane 0 refills its own stages between compute steps.)
 //   * Two CTAs per SM (shared-memory carveout at its maximum) keep
-//     2 x NW x SW pages -- about 192 KB -- in flight per SM, which is what
+//     2 x NW x SW stages -- 192 KB -- in flight per SM, which is what
 //     Little's law asks for at full HBM bandwidth.
 //   * A key row is split over LPR = D/16 lanes (16 elements, two 16-byte
 //     vectors each), so a warp covers 32/LPR rows per instruction and a dot

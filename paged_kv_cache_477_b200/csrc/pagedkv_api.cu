@@ -90,23 +90,24 @@ bool make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* d
 
 // ----------------------------------------------------------------- decode --
 constexpr int kDecodeWarps = 4;
-// pages per ring stage: one 8 KB page pair at D=128, two at D=64, so a stage
-// is 32 key rows whenever a page is smaller and a lane always works on four
-// rows per step
-constexpr int pages_per_stage(int D) { return D == 128 ? 1 : 2; }
-// stages per warp: 96 KB of pages in flight per CTA, two CTAs per SM
-constexpr int kDecodeStages = 3;
-
-// D=64 pages are 2 KB: twice the copies per byte, issued by producer warps
-constexpr bool decode_producers(int D) { return D == 64; }
+// Pages per ring stage and stages per warp, from B200 sweeps of the three
+// decode workloads: D=128 one 8 KB page pair per stage, three stages; D=64
+// three page pairs (48 key rows, 12 KB) per stage, two stages.  Either way
+// 96 KB of pages are in flight per CTA, two CTAs per SM.  (D=64 with one page
+// pair and six stages: 8 % slower; two pairs and three stages: 3 % slower.)
+constexpr int pages_per_stage(int D) { return D == 128 ? 1 : 3; }
+constexpr int decode_stages(int D) { return D == 128 ? 3 : 2; }
+// Copies are issued by producer warps, one per consumer warp (at D=64, twice
+// the copies per byte: 3.78 -> 4.08 TB/s; at D=128 0.6-1.6 % faster).
+constexpr bool decode_producers(int) { return true; }
 
 template <int D, int HG>
-using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D), decode_producers(D)>;
+using DecodeS = pkv::DecodeShape<D, HG, kDecodeWarps, decode_stages(D), pages_per_stage(D), decode_producers(D)>;
 
 template <int D, int HG, bool WIN = false>
 struct DecodeKernel {
   static constexpr auto fn =
-      pkv::decode_attn_kernel<D, HG, kDecodeWarps, kDecodeStages, pages_per_stage(D), WIN, decode_producers(D)>;
+      pkv::decode_attn_kernel<D, HG, kDecodeWarps, decode_stages(D), pages_per_stage(D), WIN, decode_producers(D)>;
   // set the dynamic shared-memory limit once per device; return CTAs per SM
   static int prepare(int dev) {
     static int occ[kMaxDevices] = {0};
