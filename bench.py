@@ -50,7 +50,7 @@ def parse():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--profile", default=None,
-                    choices=["decode", "decode_full", "decode_d64", "decode_int8", "decode_int8_full", "split", "prefill",
+                    choices=["decode", "decode_full", "decode_d64", "decode_gqa8", "decode_int8", "decode_int8_full", "split", "prefill",
                              "write"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
@@ -405,7 +405,7 @@ def extras(peaks, decode_gbs):
                      "l2": "new rows warm in L2; rows scattered into a 2 GiB pool"}
     del c
     torch.cuda.empty_cache()
-    for name, hint in (("llama32_1b_decode", 4096), ("ragged_long_decode", 32768)):
+    for name, hint in (("llama32_1b_decode", 4096), ("ragged_long_decode", 32768), ("gqa8_decode", 4096)):
         c = wl.workload(name, device="cuda")
         out = torch.empty_like(c.q)
         ws = torch.empty(max(1, pkv.workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, hint)),
@@ -551,6 +551,13 @@ def profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
                                 max_context_len=4096, workspace=ws)
+    elif kind == "decode_gqa8":
+        # eight query heads per kv head (64 q / 8 kv heads, D=128, ctx 4096): 1 GiB of K/V
+        c = wl.workload("gqa8_decode", device="cuda")
+        out = torch.empty_like(c.q)
+        for _ in range(launches):
+            pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
+                                max_context_len=4096)
     elif kind == "decode_d64":
         # the Llama-3.2-1B-shaped decode (D=64): 300 MB of K/V
         c = wl.workload("llama32_1b_decode", device="cuda")

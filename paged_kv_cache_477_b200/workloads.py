@@ -198,7 +198,8 @@ def make_case(*, name: str = "custom", kind: str = "decode", B: int, Hq: int, Hk
 
 
 # --------------------------------------------------------------------------- #
-# The five named workloads.                                                    #
+# The named workloads (the five of the measurement plan, their INT8 and
+# eight-heads-per-group variants).                                                    #
 # --------------------------------------------------------------------------- #
 
 def _lens_llama32_1b(seed: int):
@@ -237,6 +238,10 @@ WORKLOADS = {
         kind="decode", B=16, Hq=32, Hkv=8, D=128, bs=16, lens=_lens_ragged(1004), seed=1004,
         desc="ragged long-context decode: B=16, Hq=32/Hkv=8, D=128, 4 x 32768 + 12 log-uniform "
              "[128, 8192]"),
+    "gqa8_decode": dict(
+        kind="decode", B=64, Hq=64, Hkv=8, D=128, bs=16, lens=[4096] * 64, seed=1007,
+        desc="grouped-query decode with eight query heads per kv head: B=64, Hq=64/Hkv=8, D=128, bs=16, "
+             "ctx 4096"),
     "chunked_prefill": dict(
         kind="prefill", B=4, Hq=32, Hkv=8, D=128, bs=16, lens=[4096] * 4, q_len=[512] * 4,
         seed=1005, pool_blocks=1024,

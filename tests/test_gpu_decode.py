@@ -169,6 +169,34 @@ def test_decode_ragged_long_workload_full():
     _no_device_error()
 
 
+def test_decode_gqa8_workload_full():
+    """Eight query heads per kv head (64 q / 8 kv heads, D=128, ctx 4096): one
+    CTA takes the whole group, so each page is read once; every row against
+    the oracle."""
+    case = wl.workload("gqa8_decode", device="cuda")
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale, max_context_len=4096)
+    assert_close(out, HostCase(case).decode_ref(), "gqa8_decode")
+    _no_device_error()
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_gqa8_split_and_window(D):
+    """Eight heads per kv head through explicit splits and a sliding window,
+    ragged lengths with empty and partial pages."""
+    case = _decode_case([3000, 1, 0, 517, 2048, 33], 32, 4, D, seed=90 + D)
+    ref = HostCase(case).decode_ref()
+    for pps in (1, 7, 64):
+        out = pkv.paged_attention_split(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                        case.context_lens, case.scale, pages_per_split=pps)
+        assert_close(out, ref, f"gqa8 split pps={pps} D={D}")
+    for window in (1, 100, 1000):
+        out = pkv.paged_attention_window(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                         case.context_lens, case.scale, window)
+        assert_close(out, HostCase(case).decode_window_ref(window), f"gqa8 window={window} D={D}")
+    _no_device_error()
+
+
 def test_split_count_invariance():
     case = _decode_case([2000, 37, 900, 1], 8, 2, 128, seed=9)
     ref = HostCase(case).decode_ref()
