@@ -295,7 +295,7 @@ pkv_status pkv_paged_attention_split_noalloc(
  *   q               : device, [sumQ][Hq][D] bf16
  *   query_start_loc : device, [B+1] int32, query_start_loc[0] = 0
  *   max_q_len       : host upper bound on Q_b (sizes the launch)
- * Needs D in {64, 128}, bs = 16, Hq / Hkv dividing 128 (else
+ * Needs D in {64, 128}, bs = 16, Hq / Hkv <= 128 (else
  * PKV_ERR_UNSUPPORTED); scale may have either sign but must be finite (else
  * PKV_ERR_INVALID_ARG).
  */

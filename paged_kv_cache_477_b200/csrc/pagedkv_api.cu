@@ -785,7 +785,7 @@ pkv_status prefill_impl(void* out, const void* q, const int32_t* query_start_loc
     return PKV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
-  if ((D != 64 && D != 128) || bs != pkv::kPageRows || G > pkv::pf::BM || pkv::pf::BM % G != 0)
+  if ((D != 64 && D != 128) || bs != pkv::kPageRows || G > pkv::pf::BM)
     return PKV_ERR_UNSUPPORTED;
   if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
   if (B == 0 || sumQ == 0 || max_q_len == 0) return PKV_OK;

@@ -13,7 +13,9 @@
 // B200 design (one CTA per SM, 12 warps):
 //   * A CTA owns a task: two 128-row query tiles of one (sequence, kv head).
 //     The G query heads of the kv head are packed into the rows (row =
-//     position * G + head), so every K/V tile loaded feeds 256 query rows.
+//     position * G + head), so every K/V tile loaded feeds 256 query rows;
+//     a tile holds floor(128 / G) whole positions (when G does not divide
+//     128 its last rows stay idle).
 //     The tasks of one (sequence, kv head) are consecutive in the grid, so
 //     they run in the same wave and its K/V pages cross HBM once.
 //   * Warp 0 (lanes 0-7) loads Q once and the K tiles of 128 keys (eight
@@ -314,7 +316,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
       }
       const PrefillTask k = prefill_task<WIN>(p);
       if (kload && lane == 0) {
-        mbar_arrive_expect_tx(bar(pf::B_Q), pf::NQT * LY::TILE_BYTES);
+        // a query tile holds PPT whole positions of G heads: G * PPT <= 128
+        // rows (the rows past them are never loaded and never written out)
+        mbar_arrive_expect_tx(bar(pf::B_Q), pf::NQT * LY::NH * 128 * G * PPT);
         for (int i = 0; i < pf::NQT; ++i) {
           const uint32_t qd = base + LY::Q_OFF + i * LY::TILE_BYTES;
           const int z = k.qs + k.p0 + i * PPT;
@@ -472,7 +476,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     const uint32_t masked_bits = __float_as_uint(neg ? INFINITY : -INFINITY);
     const PrefillTask k = prefill_task<WIN>(p);
     const int pos = k.p0 + qt * PPT + r / G, hh = r % G;
-    const bool row_valid = pos < k.Qb;
+    const bool row_valid = r < PPT * G && pos < k.Qb;
     const int limit = k.L - k.Qb + min(pos, k.Qb - 1);  // last key this row may see
     const int lo = WIN ? limit - p.window + 1 : 0;  // first key this row may see
     float m_run = -INFINITY, l_run = 0.f;

@@ -107,12 +107,27 @@ def test_prefill_rejects_unsupported_shapes_and_bad_scales():
                                         case.block_tables, case.context_lens, scale, case.max_q_len)
         assert e.value.status == status
         assert pkv.last_launch_count() == 0
-    odd = _prefill_case([32], [16], 12, 4, seed=604)        # 3 query heads per kv head: 3 does not divide 128
+    wide = _prefill_case([32], [16], 129, 1, seed=604)      # 129 query heads per kv head: more than a tile
     with pytest.raises(pkv.PagedKVError) as e:
-        pkv.paged_attention_prefill(odd.q, odd.query_start_loc, odd.k_cache, odd.v_cache, odd.block_tables,
-                                    odd.context_lens, odd.scale, odd.max_q_len)
+        pkv.paged_attention_prefill(wide.q, wide.query_start_loc, wide.k_cache, wide.v_cache, wide.block_tables,
+                                    wide.context_lens, wide.scale, wide.max_q_len)
     assert e.value.status == 2
     assert pkv.last_launch_count() == 0
+
+
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("Hq,Hkv", [(12, 4), (6, 2), (10, 2), (7, 1), (24, 2)])
+def test_prefill_group_sizes_not_dividing_128(Hq, Hkv, D):
+    """Groups of 3, 5, 7 and 12 query heads: a tile holds floor(128 / G) whole
+    positions and its last rows stay idle; chunks across several tiles,
+    partial last pages."""
+    lens = [300, 77, 129, 45]
+    qlens = [130, 77, 1, 45]
+    case = _prefill_case(lens, qlens, Hq, Hkv, seed=700 + Hq + D, D=D)
+    out, host = _run(case)
+    ref, tok = host.prefill_ref()
+    assert_close(out[tok], ref, f"prefill G={Hq // Hkv} D={D}")
+    assert pkv.get_device_error() == 0
 
 
 @pytest.mark.parametrize("D", [128, 64])
