@@ -436,9 +436,26 @@ __global__ void __launch_bounds__(NW * 32 * (PROD ? 2 : 1), PROD ? 2 : 1)
     int blk[PPS];
 #pragma unroll
     for (int i = 0; i < PPS; ++i) blk[i] = __shfl_sync(0xffffffffu, bt_cur.blk[i], k & 31);
-    if (lane == 0) {
-      const int s = k % SW;
-      const uint32_t stage = wring + s * S::STAGE_BYTES;
+    const int s = k % SW;
+    const uint32_t stage = wring + s * S::STAGE_BYTES;
+    if (PROD) {
+      // A thread issues bulk copies at a fixed rate whatever their size, so
+      // the producer spreads a stage's 2 np copies over as many lanes: lane i
+      // copies K page i, lane np + i V page i.  The byte count is posted first.
+      if (lane == 0) mbar_arrive_expect_tx(wbar + 8 * s, np * 2 * S::PAGE_BYTES);
+      __syncwarp();
+      if (lane < 2 * np) {
+        const int i = lane < np ? lane : lane - np;
+        int bi = blk[0];
+#pragma unroll
+        for (int t = 1; t < PPS; ++t)
+          if (i == t) bi = blk[t];
+        const size_t off = ((size_t)bi * p.Hkv + kvh) * S::PAGE_BYTES;
+        const bool is_k = lane < np;
+        bulk_g2s_hint(stage + (is_k ? i : PPS + i) * S::PAGE_BYTES, (is_k ? p.k_cache : p.v_cache) + off,
+                      S::PAGE_BYTES, wbar + 8 * s, pol);
+      }
+    } else if (lane == 0) {
       mbar_arrive_expect_tx(wbar + 8 * s, np * 2 * S::PAGE_BYTES);
 #pragma unroll
       for (int i = 0; i < PPS; ++i) {

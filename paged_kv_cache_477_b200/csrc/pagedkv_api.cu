@@ -95,8 +95,14 @@ constexpr int kDecodeWarps = 4;
 // three page pairs (48 key rows, 12 KB) per stage, two stages.  Either way
 // 96 KB of pages are in flight per CTA, two CTAs per SM.  (D=64 with one page
 // pair and six stages: 8 % slower; two pairs and three stages: 3 % slower.)
-constexpr int pages_per_stage(int D) { return D == 128 ? 1 : 3; }
-constexpr int decode_stages(int D) { return D == 128 ? 3 : 2; }
+#ifndef PKV_DECODE_PPS64
+#define PKV_DECODE_PPS64 3
+#endif
+#ifndef PKV_DECODE_STAGES64
+#define PKV_DECODE_STAGES64 2
+#endif
+constexpr int pages_per_stage(int D) { return D == 128 ? 1 : PKV_DECODE_PPS64; }
+constexpr int decode_stages(int D) { return D == 128 ? 3 : PKV_DECODE_STAGES64; }
 // Copies are issued by producer warps, one per consumer warp (at D=64, twice
 // the copies per byte: 3.78 -> 4.08 TB/s; at D=128 0.6-1.6 % faster).
 constexpr bool decode_producers(int) { return true; }
