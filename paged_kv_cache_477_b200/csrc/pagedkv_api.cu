@@ -186,8 +186,14 @@ size_t split_ws_bytes(int32_t B, int32_t Hq, int32_t D, int32_t C) {
 // long enough to leave one CTA running alone at the end: splits of up to
 // kSplitPagesMany pages then.  The host sees only max_context_len, not the
 // lengths themselves, so the rule is written for the longest context.
-constexpr int kSplitPages = 96;
-constexpr int kSplitPagesMany = 256;
+#ifndef PKV_SPLIT_PAGES
+#define PKV_SPLIT_PAGES 96
+#endif
+#ifndef PKV_SPLIT_PAGES_MANY
+#define PKV_SPLIT_PAGES_MANY 256
+#endif
+constexpr int kSplitPages = PKV_SPLIT_PAGES;
+constexpr int kSplitPagesMany = PKV_SPLIT_PAGES_MANY;
 constexpr int kWavesNoSplit = 3;
 
 DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, int32_t bs,
