@@ -197,6 +197,29 @@ def test_decode_gqa8_split_and_window(D):
     _no_device_error()
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("scale", [-0.125, -1.0])
+def test_decode_negative_scale(D, scale):
+    """A negative scale reverses the score order; one CTA per head group, explicit
+    splits and a sliding window, against the oracle (pinned for negative scales)."""
+    lens = [3000, 1, 0, 517, 2048, 33]
+    pages = sum(-(-L // 16) for L in lens)
+    case = wl.make_case(B=len(lens), Hq=16, Hkv=4, D=D, bs=16, lens=lens, seed=95 + D, device="cuda",
+                        pool_blocks=pages + 3, scale=scale)
+    host = HostCase(case)
+    ref = host.decode_ref()
+    out = pkv.paged_attention(case.q, case.k_cache, case.v_cache, case.block_tables, case.context_lens,
+                              case.scale)
+    assert_close(out, ref, f"negative scale {scale} D={D}")
+    out = pkv.paged_attention_split(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                    case.context_lens, case.scale, pages_per_split=7)
+    assert_close(out, ref, f"negative scale {scale} D={D} split")
+    out = pkv.paged_attention_window(case.q, case.k_cache, case.v_cache, case.block_tables,
+                                     case.context_lens, case.scale, 100)
+    assert_close(out, host.decode_window_ref(100), f"negative scale {scale} D={D} window")
+    _no_device_error()
+
+
 def test_split_count_invariance():
     case = _decode_case([2000, 37, 900, 1], 8, 2, 128, seed=9)
     ref = HostCase(case).decode_ref()

@@ -138,6 +138,19 @@ def test_int8_decode_query_dynamic_range(D):
     assert pkv.get_device_error() == 0
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_int8_decode_negative_scale(D):
+    """A negative scale over the INT8 cache (the integer scores are scaled after
+    the tensor-core product), plain and split, against the oracle."""
+    lens = [5000, 3, 0, 17, 1200, 640]
+    pages = sum(-(-L // 16) for L in lens)
+    case = wl.make_case(B=len(lens), Hq=16, Hkv=4, D=D, bs=16, lens=lens, seed=215 + D, device="cuda",
+                        pool_blocks=pages + 3, kv_dtype="int8", scale=-0.2)
+    ref = HostCase(case).decode_ref()
+    assert_close(_decode(case), ref, f"int8 negative scale D={D}")
+    assert pkv.get_device_error() == 0
+
+
 def test_int8_decode_long_contexts_split():
     """Contexts long enough for the automatic plan to split (partials + merge)."""
     case = _case([5000, 3, 0, 17, 1200, 4096, 640, 33] * 2, 32, 8, 128, seed=210)
