@@ -582,15 +582,39 @@ __global__ void __launch_bounds__(D) lse_merge_kernel(const __grid_constant__ Me
   const size_t row = (size_t)b * p.Hq + h;
   const float* lse = p.lse_part + row * p.num_splits;
   const float* o = p.o_part + row * p.num_splits * D;
+  // Loads are issued MU splits at a time (a long context has tens of splits;
+  // one dependent load per split would serialise their latencies).  Every
+  // split below nval holds at least one page and wrote its partial (o = 0 and
+  // lse = -inf when a window masked all its rows).
+  constexpr int MU = 8;
   float M = -INFINITY;
-  for (int c = 0; c < nval; ++c) M = fmaxf(M, lse[c]);
-  float ws = 0.f, a = 0.f;
-  for (int c = 0; c < nval; ++c) {
-    if (lse[c] == -INFINITY) continue;
-    const float w = ex2(lse[c] - M);
-    ws += w;
-    a = fmaf(w, o[(size_t)c * D + d], a);
+  int c = 0;
+  for (; c + MU <= nval; c += MU) {
+    float l8[MU];
+#pragma unroll
+    for (int i = 0; i < MU; ++i) l8[i] = lse[c + i];
+#pragma unroll
+    for (int i = 0; i < MU; ++i) M = fmaxf(M, l8[i]);
   }
+  for (; c < nval; ++c) M = fmaxf(M, lse[c]);
+  float ws = 0.f, a = 0.f;
+  auto add = [&](float lc, float oc) {
+    const float w = lc == -INFINITY ? 0.f : ex2(lc - M);
+    ws += w;
+    a = fmaf(w, oc, a);
+  };
+  c = 0;
+  for (; c + MU <= nval; c += MU) {
+    float l8[MU], o8[MU];
+#pragma unroll
+    for (int i = 0; i < MU; ++i) {
+      l8[i] = lse[c + i];
+      o8[i] = o[(size_t)(c + i) * D + d];
+    }
+#pragma unroll
+    for (int i = 0; i < MU; ++i) add(l8[i], o8[i]);
+  }
+  for (; c < nval; ++c) add(lse[c], o[(size_t)c * D + d]);
   p.out[row * D + d] = __float2bfloat16_rn(ws > 0.f ? a / ws : 0.f);
 }
 

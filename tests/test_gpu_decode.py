@@ -116,8 +116,11 @@ EDGE_LENS = [0, 1, 15, 16, 17, 31, 32, 33, 100, 257, 600]
 
 
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2), (8, 2), (16, 2), (6, 2), (32, 8), (16, 8), (24, 12), (8, 8)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2), (8, 2), (16, 2), (6, 2), (32, 8), (16, 8), (24, 12), (8, 8),
+                                    (3, 3), (6, 3), (12, 3), (4, 1)])
 def test_decode_shapes_and_edges(D, Hq, Hkv):
+    """Query heads per kv head from 1 to 8 (dividing 4 or not), odd and even kv-head
+    counts, at both head sizes; ragged lengths from empty to several pages."""
     case = _decode_case(EDGE_LENS, Hq, Hkv, D, seed=100 + D + Hq)
     host = HostCase(case)
     ref = host.decode_ref()
