@@ -493,6 +493,20 @@ def extras(peaks, decode_gbs):
                                      "l2": "inputs larger than L2"}
     del c, out, ws
     torch.cuda.empty_cache()
+    # INT8 cache over the ragged long-context batch (split-KV through the int8 kernel)
+    c = wl.workload("ragged_long_decode", device="cuda", kv_dtype="int8")
+    out = torch.empty_like(c.q)
+    ws = torch.empty(max(1, pkv.workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, 32768)), dtype=torch.uint8,
+                     device="cuda")
+    us = timed_us(lambda: pkv.paged_attention_int8(c.q, c.k_cache, c.v_cache, c.k_scale, c.v_scale, c.block_tables,
+                                                   c.context_lens, c.scale, out=out, max_context_len=32768,
+                                                   workspace=ws), 20)
+    res["ragged_long_decode_int8"] = {"GB/s": round(decode_bytes(c) / (us * 1e-6) / 1e9, 1), "us": round(us, 2),
+                                      "frac_hbm": round(decode_bytes(c) / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                                      "launches": pkv.last_launch_count(), "bytes": decode_bytes(c),
+                                      "l2": "inputs larger than L2"}
+    del c, out, ws
+    torch.cuda.empty_cache()
     c = wl.workload("chunked_prefill", device="cuda")
     # the prefill's pre-step: the chunk's 2048 rows into the cache
     wfn = lambda: pkv.kv_cache_write(c.new_key, c.new_value, c.k_cache, c.v_cache, c.slot_mapping)

@@ -113,8 +113,8 @@ pkv_status pkv_paged_attention(void* out, const void* q, const void* k_cache,
                                size_t workspace_bytes, pkv_dtype dtype,
                                pkv_stream_t stream);
 
-/* Workspace bytes pkv_paged_attention may use for these sizes on the current
- * device (0 if it would never split). */
+/* Workspace bytes pkv_paged_attention (or pkv_paged_attention_int8) may use
+ * for these sizes on the current device (0 if it would never split). */
 size_t pkv_paged_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv,
                                           int32_t D, int32_t MB, int32_t bs,
                                           int32_t max_context_len_hint);
@@ -167,7 +167,8 @@ pkv_status pkv_kv_cache_write_int8(const void* key, const void* value,
 
 /*
  * paged_attention_int8 -- pkv_paged_attention over the int8 cache: the same
- * split plan, workspace (pkv_paged_attention_workspace_size) and errors; K and
+ * workspace (pkv_paged_attention_workspace_size bytes serve either cache) and
+ * errors, with split sizes chosen for this kernel; K and
  * V are read as codes and scaled by their row's scale inside the kernel (half
  * the bytes of the bf16 cache, plus 4 bytes per row).  q and out are bf16 as
  * for pkv_paged_attention; D in {64, 128}, bs = 16.  The scores q.k are
@@ -326,8 +327,8 @@ pkv_status pkv_paged_attention_prefill_window(
  * L-window .. L-1, as pkv_paged_attention_window does over the bf16 cache
  * (the inference-lab page's sliding-window cache, section "KV缓存实验与长上下文
  * 优化", over the Tiny-Infer page's INT8 cache, section "推测性解码与INT8量化").
- * Same plan and workspace as pkv_paged_attention_window
- * (pkv_paged_attention_window_workspace_size); errors as
+ * Same workspace as pkv_paged_attention_window
+ * (pkv_paged_attention_window_workspace_size bytes serve either cache); errors as
  * pkv_paged_attention_int8.  Pages wholly before the window are never read.
  */
 pkv_status pkv_paged_attention_int8_window(void* out, const void* q, const void* k_cache,

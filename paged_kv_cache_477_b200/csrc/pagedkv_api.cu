@@ -194,10 +194,16 @@ size_t split_ws_bytes(int32_t B, int32_t Hq, int32_t D, int32_t C) {
 #endif
 constexpr int kSplitPages = PKV_SPLIT_PAGES;
 constexpr int kSplitPagesMany = PKV_SPLIT_PAGES_MANY;
+// The int8 cache moves half the bytes per page, so its splits are longer
+// (ragged long-context batch: 192 pages 94.6 us, 96 pages 102.7 us, 256 pages
+// 96.7 us; the Llama-3.2-1B shape is the same at every size).
+#ifndef PKV_SPLIT_PAGES_INT8
+#define PKV_SPLIT_PAGES_INT8 192
+#endif
 constexpr int kWavesNoSplit = 3;
 
 DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, int32_t bs,
-                     int32_t hint) {
+                     int32_t hint, bool int8 = false) {
   DecodePlan pl{1, std::max<int32_t>(MB, 1), 0};
   const int max_pages = max_pages_of(MB, bs, hint);
   const int G = Hq / Hkv, HG = heads_per_cta(G);
@@ -206,7 +212,7 @@ DecodePlan plan_auto(int32_t B, int32_t Hq, int32_t Hkv, int32_t D, int32_t MB, 
   const int occ = std::max(1, decode_occupancy(D, HG, dev));
   const int64_t slots = (int64_t)device_sm_count(dev) * occ;
   if (units <= 0) return pl;
-  const int target = units >= kWavesNoSplit * slots ? kSplitPagesMany : kSplitPages;
+  const int target = units >= kWavesNoSplit * slots ? kSplitPagesMany : (int8 ? PKV_SPLIT_PAGES_INT8 : kSplitPages);
   const int C = (max_pages + target - 1) / target;
   if (C <= 1) return pl;
   const int pps = (max_pages + C - 1) / C;  // equal splits no longer than the target
@@ -533,7 +539,7 @@ pkv_status pkv_paged_attention_int8(void* out, const void* q, const void* k_cach
   if (s != PKV_OK || B == 0) return s;
   if (MB > 0 && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale)))
     return PKV_ERR_INVALID_ARG;
-  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint);
+  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint, true);
   if (pl.num_splits > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned16(workspace)))
     pl = DecodePlan{1, std::max<int32_t>(MB, 1), 0};  // no room: one CTA per head group
   if (pl.num_splits == 1) pl.pages_per_split = std::max<int32_t>(MB, 1);
@@ -560,9 +566,10 @@ pkv_status pkv_paged_attention_int8_window(void* out, const void* q, const void*
   if (window < 1) return PKV_ERR_INVALID_ARG;
   if (MB > 0 && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale)))
     return PKV_ERR_INVALID_ARG;
-  // the plan of pkv_paged_attention_window: over the pages a window touches
+  // the plan of pkv_paged_attention_window (split sizes for this kernel):
+  // over the pages a window touches
   const int32_t span = (int32_t)std::min<int64_t>((int64_t)window_pages(window) * bs, (int64_t)MB * bs);
-  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, span);
+  DecodePlan pl = plan_auto(B, Hq, Hkv, D, MB, bs, span, true);
   if (pl.num_splits > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned16(workspace)))
     pl = DecodePlan{1, std::max<int32_t>(MB, 1), 0};  // no room: one CTA per head group
   if (pl.num_splits == 1) pl.pages_per_split = std::max<int32_t>(MB, 1);
@@ -598,7 +605,9 @@ size_t pkv_paged_attention_window_workspace_size(int32_t B, int32_t Hq, int32_t 
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || (D != 64 && D != 128) || bs != pkv::kPageRows || window < 1)
     return 0;
   const int32_t span = (int32_t)std::min<int64_t>((int64_t)window_pages(window) * bs, (int64_t)MB * bs);
-  return plan_auto(B, Hq, Hkv, D, MB, bs, span).workspace;
+  // enough for the bf16 and the int8 kernel's plans alike
+  return std::max(plan_auto(B, Hq, Hkv, D, MB, bs, span).workspace,
+                  plan_auto(B, Hq, Hkv, D, MB, bs, span, true).workspace);
 }
 
 pkv_status pkv_kv_cache_write_rope(const void* key, const void* value, int64_t key_stride_tok,
@@ -738,7 +747,9 @@ size_t pkv_paged_attention_workspace_size(int32_t B, int32_t Hq, int32_t Hkv, in
                                           int32_t MB, int32_t bs, int32_t max_context_len_hint) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || (D != 64 && D != 128) || bs != pkv::kPageRows)
     return 0;
-  return plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint).workspace;
+  // enough for the bf16 and the int8 kernel's plans alike
+  return std::max(plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint).workspace,
+                  plan_auto(B, Hq, Hkv, D, MB, bs, max_context_len_hint, true).workspace);
 }
 
 pkv_status pkv_paged_attention(void* out, const void* q, const void* k_cache, const void* v_cache,

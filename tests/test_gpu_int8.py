@@ -175,6 +175,17 @@ def test_int8_write_then_decode_llama3_8b_shaped_full():
     assert pkv.get_device_error() == 0
 
 
+def test_int8_decode_ragged_long_workload_full():
+    """The ragged long-context batch over the int8 cache (4 x 32768 and 12 shorter
+    contexts, split into the int8 kernel's longer splits and merged); every row
+    of the 16 sequences against the int8 oracle."""
+    case = wl.workload("ragged_long_decode", device="cuda", kv_dtype="int8")
+    out = _decode(case, max_context_len=32768)
+    assert pkv.last_launch_count() == 2                  # split partials + merge
+    assert_close(out, HostCase(case).decode_ref(), "ragged_long_decode int8")
+    assert pkv.get_device_error() == 0
+
+
 def test_int8_decode_bad_block_id_is_reported():
     case = _case([40, 40], 4, 2, 64, seed=211)
     bt = case.block_tables.clone()
