@@ -50,8 +50,8 @@ def parse():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--profile", default=None,
-                    choices=["decode", "decode_full", "decode_d64", "decode_gqa8", "decode_int8", "decode_int8_full", "split", "prefill",
-                             "write"],
+                    choices=["decode", "decode_full", "decode_d64", "decode_gqa8", "decode_ragged", "decode_int8",
+                             "decode_int8_full", "split", "prefill", "write"],
                     help="run a few launches of one kernel on a small case (for ncu) and exit")
     return ap.parse_args()
 
@@ -579,6 +579,15 @@ def profile_case(kind: str, launches: int = 3):
         for _ in range(launches):
             pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
                                 max_context_len=4096)
+    elif kind == "decode_ragged":
+        # the ragged long-context batch (4 x 32768 + 12 shorter, split-KV + merge): 620 MB of K/V
+        c = wl.workload("ragged_long_decode", device="cuda")
+        out = torch.empty_like(c.q)
+        ws = torch.empty(max(1, pkv.workspace_size(c.B, c.Hq, c.Hkv, c.D, c.MB, 16, 32768)), dtype=torch.uint8,
+                         device="cuda")
+        for _ in range(launches):
+            pkv.paged_attention(c.q, c.k_cache, c.v_cache, c.block_tables, c.context_lens, c.scale, out=out,
+                                max_context_len=32768, workspace=ws)
     elif kind == "decode_int8_full":
         # the bench's Llama-3-8B-shaped INT8 decode, full size: 1.1 GB of codes and scales
         c = wl.workload("llama3_8b_decode_int8", device="cuda")

@@ -582,39 +582,36 @@ __global__ void __launch_bounds__(D) lse_merge_kernel(const __grid_constant__ Me
   const size_t row = (size_t)b * p.Hq + h;
   const float* lse = p.lse_part + row * p.num_splits;
   const float* o = p.o_part + row * p.num_splits * D;
-  // Loads are issued MU splits at a time (a long context has tens of splits;
-  // one dependent load per split would serialise their latencies).  Every
-  // split below nval holds at least one page and wrote its partial (o = 0 and
-  // lse = -inf when a window masked all its rows).
+  // Loads are issued MU splits at a time, predicated past nval, so a
+  // sequence's splits cost two load round trips per MU of them instead of one
+  // dependent load per split.  Every split below nval holds at least one page
+  // and wrote its partial (o = 0 and lse = -inf when a window masked all its
+  // rows).
   constexpr int MU = 8;
   float M = -INFINITY;
-  int c = 0;
-  for (; c + MU <= nval; c += MU) {
+  for (int c0 = 0; c0 < nval; c0 += MU) {
     float l8[MU];
 #pragma unroll
-    for (int i = 0; i < MU; ++i) l8[i] = lse[c + i];
+    for (int i = 0; i < MU; ++i) l8[i] = c0 + i < nval ? lse[c0 + i] : -INFINITY;
 #pragma unroll
     for (int i = 0; i < MU; ++i) M = fmaxf(M, l8[i]);
   }
-  for (; c < nval; ++c) M = fmaxf(M, lse[c]);
   float ws = 0.f, a = 0.f;
-  auto add = [&](float lc, float oc) {
-    const float w = lc == -INFINITY ? 0.f : ex2(lc - M);
-    ws += w;
-    a = fmaf(w, oc, a);
-  };
-  c = 0;
-  for (; c + MU <= nval; c += MU) {
+  for (int c0 = 0; c0 < nval; c0 += MU) {
     float l8[MU], o8[MU];
 #pragma unroll
     for (int i = 0; i < MU; ++i) {
-      l8[i] = lse[c + i];
-      o8[i] = o[(size_t)(c + i) * D + d];
+      const bool in = c0 + i < nval;
+      l8[i] = in ? lse[c0 + i] : -INFINITY;
+      o8[i] = in ? o[(size_t)(c0 + i) * D + d] : 0.f;
     }
 #pragma unroll
-    for (int i = 0; i < MU; ++i) add(l8[i], o8[i]);
+    for (int i = 0; i < MU; ++i) {
+      const float w = l8[i] == -INFINITY ? 0.f : ex2(l8[i] - M);
+      ws += w;
+      a = fmaf(w, o8[i], a);
+    }
   }
-  for (; c < nval; ++c) add(lse[c], o[(size_t)c * D + d]);
   p.out[row * D + d] = __float2bfloat16_rn(ws > 0.f ? a / ws : 0.f);
 }
 
