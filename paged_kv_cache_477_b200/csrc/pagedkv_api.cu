@@ -17,6 +17,7 @@
 #include "block_allocator.hpp"
 #include "decode_attn.cuh"
 #include "decode_attn_i8.cuh"
+#include "lse_merge.cuh"
 #include "hbm_probe.cuh"
 #include "kv_cache_write.cuh"
 #include "pkv_common.cuh"
