@@ -376,6 +376,16 @@ __global__ void __launch_bounds__(NW * 32 * (PROD ? 2 : 1), PROD ? 2 : 1)
   }
   const int npages = (L + kPageRows - 1) / kPageRows;
   const int n = min(npages - pg0, p.pages_per_split);  // pages of this CTA
+  if (n <= 0) {
+    // A split past the end of a shorter sequence leaves at once (a ragged
+    // batch launches many); with one split only an empty context reaches
+    // here, and its output is zero.  (In split mode the merge counts the
+    // non-empty splits itself.)
+    if (p.num_splits == 1)
+      for (int i = threadIdx.x; i < HG * D; i += blockDim.x)
+        p.out[((size_t)b * p.Hq + head0 + i / D) * D + i % D] = __float2bfloat16_rn(0.f);
+    return;
+  }
   // A wait that ran out earlier leaves a sticky error: do no more work until
   // the host has read and cleared it.  One thread reads the word so the whole
   // CTA takes the same branch.
@@ -383,14 +393,6 @@ __global__ void __launch_bounds__(NW * 32 * (PROD ? 2 : 1), PROD ? 2 : 1)
   if (threadIdx.x == 0) s_stop = *reinterpret_cast<volatile int*>(&g_error_word) == PKV_ERR_TIMEOUT;
   __syncthreads();
   if (s_stop) return;
-  if (n <= 0) {
-    // Only an empty context reaches here with one split: its output is zero.
-    // (In split mode the merge counts the non-empty splits itself.)
-    if (p.num_splits == 1)
-      for (int i = threadIdx.x; i < HG * D; i += blockDim.x)
-        p.out[((size_t)b * p.Hq + head0 + i / D) * D + i % D] = __float2bfloat16_rn(0.f);
-    return;
-  }
 
   // ------------------------------------------------ this warp's unit stream --
   const int nu = (n + PPS - 1) / PPS;                        // units of this CTA

@@ -118,16 +118,16 @@ __global__ void __launch_bounds__(DecodeI8Shape<D, HG>::THREADS)
   }
   const int npages = (L + kPageRows - 1) / kPageRows;
   const int n = min(npages - pg0, p.pages_per_split);  // pages of this CTA
-  __shared__ int s_stop;
-  if (threadIdx.x == 0) s_stop = *reinterpret_cast<volatile int*>(&g_error_word) == PKV_ERR_TIMEOUT;
-  __syncthreads();
-  if (s_stop) return;
-  if (n <= 0) {
+  if (n <= 0) {  // a split past the sequence's end leaves at once; an empty context writes zeros
     if (p.num_splits == 1)
       for (int i = threadIdx.x; i < HG * D; i += blockDim.x)
         p.out[((size_t)b * p.Hq + head0 + i / D) * D + i % D] = __float2bfloat16_rn(0.f);
     return;
   }
+  __shared__ int s_stop;
+  if (threadIdx.x == 0) s_stop = *reinterpret_cast<volatile int*>(&g_error_word) == PKV_ERR_TIMEOUT;
+  __syncthreads();
+  if (s_stop) return;
   const int nt = (n + S::TILE_PAGES - 1) / S::TILE_PAGES;  // tiles of this CTA
 
   auto full = [&](int s) { return base + S::BAR_OFF + 8 * s; };
